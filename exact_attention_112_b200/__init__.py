@@ -1,0 +1,172 @@
+"""B200-native (sm_100a) exact scaled dot-product attention behind a C ABI.
+
+The compute lives in ``libfa.so`` (CUDA for sm_100a: TMA, tcgen05 tensor cores,
+tensor memory; see ``include/fa.h``).  This module only marshals arguments:
+it turns torch tensors into device pointers and sizes, calls the C entry point
+of the same name and raises ``FaError`` on a non-zero status.  There is no
+fallback: if the library is missing or the device is not an sm_100 GPU the
+calls fail.
+
+    import exact_attention_112_b200 as fa
+    o, lse = fa.attention_forward(q, k, v, causal=True)         # allocates o, lse
+    fa.fa_fwd(q, k, v, o, lse, causal=True, scale=None)          # caller-owned outputs
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, dO, causal=True)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
+    "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_F16", "FA_BF16", "FaError",
+    "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes",
+    "fa_status_string", "fa_device_status", "fa_debug_wait_timeout",
+    "attention_forward", "attention_backward",
+]
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_F16, FA_BF16 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libfa.so")
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {fa_status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with "
+                    "`python -m exact_attention_112_b200._build` (needs nvcc)")
+            L = ctypes.CDLL(path)
+            vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp]
+            L.fa_fwd.restype = i
+            L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+            L.fa_bwd_workspace_bytes.restype = sz
+            L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                 vp, vp, sz, vp]
+            L.fa_bwd.restype = i
+            L.fa_status_string.argtypes = [i]
+            L.fa_status_string.restype = ctypes.c_char_p
+            L.fa_device_status.argtypes = [vp]
+            L.fa_device_status.restype = i
+            L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
+            L.fa_debug_wait_timeout.restype = i
+            _lib = L
+    return _lib
+
+
+def fa_status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float16:
+        return FA_F16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    raise FaError(FA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
+
+
+def _check(status, what):
+    if status != FA_OK:
+        raise FaError(status, what)
+
+
+def fa_fwd(q, k, v, o, lse, causal=False, scale=None, key_bias=None, stream=None):
+    """Forward pass into caller-owned ``o`` [B,H,Nq,D] and ``lse`` [B,H,Nq] fp32."""
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for t in (q, k, v, o, lse) + (() if key_bias is None else (key_bias,)):
+        if not t.is_contiguous():
+            raise FaError(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be contiguous")
+    st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
+                      int(bool(causal)), float(scale), _dtype_code(q), _ptr(key_bias),
+                      _stream_ptr(stream))
+    _check(st, "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B, H, Nq, Nk, D) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, H, Nq, Nk, D))
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, causal=False, scale=None,
+           key_bias=None, stream=None):
+    """Backward pass into caller-owned dq, dk, dv, using a caller-owned workspace."""
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                      _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)), float(scale),
+                      _dtype_code(q), _ptr(key_bias), _ptr(workspace), nbytes,
+                      _stream_ptr(stream))
+    _check(st, "fa_bwd")
+
+
+def fa_device_status(stream=None) -> int:
+    return int(lib().fa_device_status(_stream_ptr(stream)))
+
+
+def fa_debug_wait_timeout(timeout_us: int, stream=None) -> int:
+    return int(lib().fa_debug_wait_timeout(int(timeout_us), _stream_ptr(stream)))
+
+
+def attention_forward(q, k, v, causal=False, scale=None, key_bias=None, stream=None):
+    """Allocate O and LSE with torch (device plumbing) and run ``fa_fwd``."""
+    import torch
+    B, H, Nq, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, causal=causal, scale=scale, key_bias=key_bias, stream=stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dO, causal=False, scale=None, key_bias=None,
+                       stream=None):
+    """Allocate dq, dk, dv and the workspace with torch and run ``fa_bwd``."""
+    import torch
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws = torch.empty(fa_bwd_workspace_bytes(B, H, Nq, Nk, D), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, causal=causal, scale=scale,
+           key_bias=key_bias, stream=stream)
+    return dq, dk, dv

@@ -1,0 +1,223 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
+// validation, TMA tensor-map construction, the per-device error word and the
+// launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+#include "fa_ptx.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+// One error word per device; kernels latch a code into it, fa_device_status()
+// reads and clears it.
+__device__ int g_fa_error_word;
+
+std::mutex g_mu;
+int *g_err_ptr[kMaxDevices] = {};
+int g_cc_major[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (*dev < 0 || *dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+// Per-device set-up, done once: the error word's device address and the
+// compute capability.
+int device_setup(int dev, int **err_ptr) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FA_ERR_CUDA;
+        g_cc_major[dev] = prop.major;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_fa_error_word) != cudaSuccess) return FA_ERR_CUDA;
+        g_err_ptr[dev] = static_cast<int *>(ptr);
+    }
+    if (g_cc_major[dev] != 10) return FA_ERR_UNSUPPORTED;
+    *err_ptr = g_err_ptr[dev];
+    return FA_OK;
+}
+
+int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_encode) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || p == nullptr)
+            return FA_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    *fn = g_encode;
+    return FA_OK;
+}
+
+// 3-D map over a [B*H, N, D] 16-bit tensor: box = 64 values x box_rows rows,
+// 128-byte swizzle (matches the MMA operand layout); rows past N read as 0
+// and are not written by stores.
+int make_map(CUtensorMap *m, const void *ptr, bool bf16, int D, int N, long long BH, int box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int st = get_encoder(&enc);
+    if (st != FA_OK) return st;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                     const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared shape/scalar validation of forward and backward.
+int check_common(int B, int H, int Nq, int Nk, int D, int causal, float scale, int dtype) {
+    if (B < 1 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    // every index the kernels form must fit in 32-bit signed arithmetic
+    const long long BH = static_cast<long long>(B) * H;
+    const long long units = BH * ((static_cast<long long>(Nq) + 255) / 256);
+    if (BH > INT32_MAX || units > INT32_MAX || BH * Nq > INT32_MAX) return FA_ERR_INVALID_ARG;
+    if (Nq > (1 << 30) || Nk > (1 << 30)) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim, dtype or device";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+        case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a device-side wait gave up";
+        case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: backward workspace missing or too small";
+        default: return "unknown fa_status";
+    }
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int Nq,
+           int Nk, int D, int causal, float scale, int dtype, const float *key_bias, void *stream) {
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (Nq == 0) return FA_OK;
+    if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (key_bias && !aligned16(key_bias)))
+        return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    const long long BH = static_cast<long long>(B) * H;
+    if (Nk == 0) {
+        return fa::launch_fwd_empty(o, lse, static_cast<size_t>(BH) * Nq, D, bf16, s) == cudaSuccess
+                   ? FA_OK : FA_ERR_CUDA;
+    }
+    fa::FwdTensorMaps tm;
+    if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.o, o, bf16, D, Nq, BH, 32)) != FA_OK) return st;
+    fa::FwdParams p;
+    p.B = B;
+    p.H = H;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.n_mblocks = (Nq + 255) / 256;
+    p.causal_off = Nk - Nq;
+    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    p.bias = key_bias;
+    p.lse = lse;
+    p.err = err;
+    p.timeout_ns = kDefaultTimeoutNs;
+    cudaError_t e = fa::launch_fwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
+    (void)Nk;
+    if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128)) return 0;
+    const size_t rows = static_cast<size_t>(B) * H * Nq;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return up(rows * sizeof(float)) + up(rows * D * sizeof(float)) + 256;
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
+           int causal, float scale, int dtype, const float *key_bias, void *workspace,
+           size_t workspace_bytes, void *stream) {
+    (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dO; (void)dq; (void)dk; (void)dv;
+    (void)B; (void)H; (void)Nq; (void)Nk; (void)D; (void)causal; (void)scale; (void)dtype;
+    (void)key_bias; (void)workspace; (void)workspace_bytes; (void)stream;
+    return FA_ERR_UNSUPPORTED;
+}
+
+int fa_device_status(void *stream) {
+    int dev;
+    int st = current_device(&dev);
+    if (st != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_fa_error_word, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return word;
+}
+
+}  // extern "C"
+
+// ---- bounded-wait self-test: one warp waits on a barrier nothing completes.
+namespace {
+__global__ void fa_wait_timeout_kernel(int *err, unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        fa::mbar_init(fa::smem_u32(&bar), 1);
+        fa::fence_mbar_init();
+    }
+    __syncthreads();
+    fa::WaitCtx w{timeout_ns, err, &abort_flag};
+    fa::mbar_wait(fa::smem_u32(&bar), 0, w);   // no arrive ever comes
+    __syncthreads();
+    if (threadIdx.x == 0) fa::mbar_arrive(fa::smem_u32(&bar));   // leave the barrier complete
+}
+}  // namespace
+
+extern "C" int fa_debug_wait_timeout(unsigned timeout_us, void *stream) {
+    int dev;
+    int st = current_device(&dev);
+    if (st != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    if (timeout_us == 0 || timeout_us > 10000000u) return FA_ERR_INVALID_ARG;
+    fa_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        err, static_cast<unsigned long long>(timeout_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}

@@ -1,0 +1,506 @@
+// fa_fwd.cu -- fused exact-attention forward for sm_100a (B200).
+//
+// What it computes: O = softmax(scale * Q K^T + mask) V and the row
+// log-sum-exp, as defined on the FlashAttention case-study slides
+// (nmj0.github.io, "Attention is where tokens meet"), organised as on the
+// slide "FlashAttention: the idea": Q, K, V are cut into tiles that fit on
+// chip, QK^T, mask, softmax and .V of a tile run in one kernel, and neither S
+// nor P is ever written to device memory.  Tiles are combined with the running
+// (m, l, o) update of "Online softmax: divide once, at the end"; O = o / l is
+// formed once per row after the last tile.
+//
+// B200 mapping (one CTA = one work unit of 256 query rows = two 128-row tiles
+// Q0, Q1 of one (batch, head)):
+//   * TMA streams Q once and K_j / V_j through a 2-stage shared-memory ring,
+//     handing each stage over with an mbarrier (expect_tx / complete_tx).
+//   * One thread issues tcgen05.mma: S_i = Q_i K_j^T (both operands from
+//     shared memory, fp32 accumulator in tensor memory) and O_i += P_i V_j
+//     (P_i read from tensor memory, V_j from shared memory).
+//   * Two softmax warpgroups (one per Q tile, one thread per query row) read
+//     S_i from tensor memory, apply scale and mask in the base-2 domain
+//     (qk_scale = scale * log2(e), the constant derived in "Mastering
+//     FlashAttention: The Algebraic Foundation"), update the row max and sum in
+//     registers, write P_i back into the same tensor-memory columns as 16-bit
+//     values and signal the MMA thread.  While one warpgroup works on S_0 the
+//     tensor core computes S_1, and vice versa.
+//   * Lazy rescale: the reference maximum m_ref of a row only moves when a new
+//     tile's maximum exceeds it by more than kTau (log2 units); only then are
+//     l and the O accumulator multiplied by alpha = 2^(m_ref_old - m_ref_new).
+//     Exactness rests on the slide's identity e^(s - m_old) e^(m_old - m_new)
+//     = e^(s - m_new): l, o and the final LSE all use the same m_ref.
+//   * Causal: key tiles entirely above the diagonal are never loaded or
+//     multiplied; tiles crossing it are masked per element.
+//
+// Tensor memory (512 columns x 128 lanes of 32 bits; lane = query row):
+//   cols [0,128)        S_0 (fp32), later P_0 (16-bit pairs) in cols [0,64)
+//   cols [128,256)      S_1 / P_1
+//   cols [256,256+D)    O_0 accumulator (fp32)
+//   cols [256+D,256+2D) O_1 accumulator
+// Shared memory: Q_0, Q_1 (reused as O staging for the TMA store), K ring x2,
+// V ring x2, mbarriers.
+//
+// Warp roles (10 warps): 0-3 softmax of Q_0, 4-7 softmax of Q_1, 8 TMA
+// producer, 9 MMA issuer (also allocates tensor memory).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "fa_internal.h"
+#include "fa_ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;            // query rows per tensor-core tile
+constexpr int kBN = 128;            // keys per tile
+constexpr int kThreads = 320;       // 10 warps
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kStages = 2;
+constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+struct FwdLayout {
+    static constexpr int kTileBytes = kBM * D * 2;       // one 128-row 16-bit tile
+    static constexpr int kChunkBytes = kBM * 128;        // 128 rows x 64 values
+    static constexpr int kQ = 0;                         // 2 tiles
+    static constexpr int kK = kQ + 2 * kTileBytes;       // kStages tiles
+    static constexpr int kV = kK + kStages * kTileBytes; // kStages tiles
+    static constexpr int kBar = kV + kStages * kTileBytes;
+    // barrier indices
+    static constexpr int kQFull = 0;
+    static constexpr int kKFull = 1;     // +stage
+    static constexpr int kKEmpty = 3;    // +stage
+    static constexpr int kVFull = 5;     // +stage
+    static constexpr int kVEmpty = 7;    // +stage
+    static constexpr int kSFull = 9;     // +tile
+    static constexpr int kPFull = 11;    // +tile
+    static constexpr int kOFull = 13;    // +tile
+    static constexpr int kDrain = 15;
+    static constexpr int kNumBars = 16;
+    static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;       // room to align the base
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+};
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (BF16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&h);
+    } else {
+        __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+              const FwdParams p) {
+    using L = FwdLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: heaviest (last) query blocks first so that the hardware
+    // block scheduler hands the long causal units out early.
+    const int BH = p.B * p.H;
+    const int unit = blockIdx.x;
+    const int mb = (p.n_mblocks - 1) - unit / BH;
+    const int bh = unit % BH;
+    const int m0 = mb * 2 * kBM;
+    const int n_kv_all = (p.Nk + kBN - 1) / kBN;
+    int n_kv = n_kv_all;
+    if (CAUSAL) {
+        const int last_row = min(m0 + 2 * kBM - 1, p.Nq - 1);
+        const int lim = last_row + p.causal_off;
+        n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kBN + 1);
+    }
+
+    // ---- set-up
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(L::kQFull), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(L::kKFull + s), 1);
+            mbar_init(bar(L::kKEmpty + s), 1);
+            mbar_init(bar(L::kVFull + s), 1);
+            mbar_init(bar(L::kVEmpty + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(L::kSFull + i), 1);
+            mbar_init(bar(L::kPFull + i), 4 * 32);
+            mbar_init(bar(L::kOFull + i), 1);
+        }
+        mbar_init(bar(L::kDrain), 1);
+        fence_mbar_init();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_o);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
+
+    if (warp == kProducerWarp) {
+        // ===================== TMA producer =====================
+        if (lane == 0 && n_kv > 0) {
+            int issued = 0;
+            bool ok = true;
+            mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTileBytes);
+            for (int i = 0; i < 2; ++i)
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &tm_q,
+                                bar(L::kQFull), c * 64, m0 + i * kBM, bh);
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!mbar_wait(bar(L::kKEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
+                mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sbase + L::kK + s * L::kTileBytes + c * L::kChunkBytes, &tm_k,
+                                bar(L::kKFull + s), c * 64, j * kBN, bh);
+                if (!mbar_wait(bar(L::kVEmpty + s), ph ^ 1, wctx)) { ok = false; issued = 2 * j + 1; break; }
+                mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTileBytes);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sbase + L::kV + s * L::kTileBytes + c * L::kChunkBytes, &tm_v,
+                                bar(L::kVFull + s), c * 64, j * kBN, bh);
+                issued = 2 * j + 2;
+            }
+            if (!ok) {
+                // Give the copies already in flight a bounded chance to land
+                // before the CTA (and its shared memory) goes away.
+                WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
+                volatile int zero = 0;
+                drain.abort_flag = &zero;
+                mbar_wait(bar(L::kQFull), 0, drain);
+                for (int t = (issued > 4 ? issued - 4 : 0); t < issued; ++t) {
+                    const int j = t >> 1;
+                    const int s = j & 1;
+                    const uint32_t ph = (j >> 1) & 1;
+                    mbar_wait(bar(((t & 1) ? L::kVFull : L::kKFull) + s), ph, drain);
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ===================== MMA issuer (one thread) =====================
+        if (lane == 0 && n_kv > 0) {
+            constexpr uint32_t idesc_qk = idesc_f16_f32acc(BF16, kBM, kBN, false, false);
+            constexpr uint32_t idesc_pv = idesc_f16_f32acc(BF16, kBM, D, false, true);
+            auto issue_s = [&](int i, int stage) {
+                const uint32_t qa = sbase + L::kQ + i * L::kTileBytes;
+                const uint32_t ka = sbase + L::kK + stage * L::kTileBytes;
+                const uint32_t d = tmem + (i ? L::kColS1 : L::kColS0);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                    umma_f16_ss(d, smem_desc_sw128(qa + off, 16, 1024),
+                                smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int i, int stage, bool acc) {
+                const uint32_t va = sbase + L::kV + stage * L::kTileBytes;
+                const uint32_t pa = tmem + (i ? L::kColS1 : L::kColS0);
+                const uint32_t d = tmem + (i ? L::kColO1 : L::kColO0);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    umma_f16_ts(d, pa + kk * 8, smem_desc_sw128(va + kk * 16 * 128, L::kChunkBytes, 1024),
+                                idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(bar(L::kQFull), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                umma_commit(bar(L::kSFull + 0));
+                issue_s(1, 0);
+                umma_commit(bar(L::kSFull + 1));
+                if (n_kv > 2) umma_commit(bar(L::kKEmpty + 0));
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                const bool more = j + 1 < n_kv;
+                const int s2 = (j + 1) & 1;
+                const uint32_t ph2 = ((j + 1) >> 1) & 1;
+                if (!mbar_wait(bar(L::kVFull + s), ph, wctx)) { ok = false; break; }
+                if (!mbar_wait(bar(L::kPFull + 0), j & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
+                issue_pv(0, s, j > 0);
+                if (more) {
+                    if (!mbar_wait(bar(L::kKFull + s2), ph2, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_s(0, s2);
+                    umma_commit(bar(L::kSFull + 0));
+                } else {
+                    umma_commit(bar(L::kOFull + 0));
+                }
+                if (!mbar_wait(bar(L::kPFull + 1), j & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
+                issue_pv(1, s, j > 0);
+                if (j + 2 < n_kv) umma_commit(bar(L::kVEmpty + s));
+                if (more) {
+                    issue_s(1, s2);
+                    umma_commit(bar(L::kSFull + 1));
+                    if (j + 3 < n_kv) umma_commit(bar(L::kKEmpty + s2));
+                } else {
+                    umma_commit(bar(L::kOFull + 1));
+                }
+            }
+            // Every issued MMA must finish before tensor memory is released.
+            umma_commit(bar(L::kDrain));
+            WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
+            volatile int zero = 0;
+            drain.abort_flag = &zero;
+            mbar_wait(bar(L::kDrain), 0, drain);
+        }
+    } else {
+        // ===================== softmax warpgroups =====================
+        const int i = warp >> 2;            // which Q tile
+        const int wq = warp & 3;            // lane quarter of tensor memory
+        const int row = wq * 32 + lane;     // row within the tile (= TMEM lane)
+        const int qrow = m0 + i * kBM + row;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t tS = tl + (i ? L::kColS1 : L::kColS0);
+        const uint32_t tO = tl + (i ? L::kColO1 : L::kColO0);
+        const float qk = p.qk_scale_log2;
+        // last key index this row may see
+        const int lim = CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1;
+        const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(bh / p.H) * p.Nk : nullptr;
+
+        float m_ref = neg_inf();   // log2 units
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int kv0 = j * kBN;
+            {
+                const bool got = mbar_wait(bar(L::kSFull + i), j & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            tc_fence_after();
+            uint32_t sr[128];
+            tmem_ld32dp_x128_wait(tS, sr);
+            float x[128];
+            if constexpr (HAS_BIAS) {
+                // x = s * qk_scale + bias * log2(e); every lane reads the same
+                // addresses, so each load is one broadcast transaction.
+                constexpr float kLog2e = 1.4426950408889634f;
+                const float *bt = bias_b + kv0;
+                if (kv0 + kBN <= p.Nk && (reinterpret_cast<uintptr_t>(bt) & 15) == 0) {
+                    const float4 *b4 = reinterpret_cast<const float4 *>(bt);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float4 bb = __ldg(b4 + c);
+                        x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, bb.x * kLog2e);
+                        x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, bb.y * kLog2e);
+                        x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, bb.z * kLog2e);
+                        x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, bb.w * kLog2e);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        const float bb = (kv0 + c < p.Nk) ? __ldg(bt + c) * kLog2e : 0.f;
+                        x[c] = fmaf(__uint_as_float(sr[c]), qk, bb);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+            }
+            if (kv0 + kBN - 1 > lim) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (kv0 + c > lim) x[c] = neg_inf();
+            }
+            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+                mx0 = fmaxf(mx0, x[c]);
+                mx1 = fmaxf(mx1, x[c + 1]);
+                mx2 = fmaxf(mx2, x[c + 2]);
+                mx3 = fmaxf(mx3, x[c + 3]);
+            }
+            float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            if constexpr (!HAS_BIAS) m_tile *= qk;   // qk > 0: max commutes with scaling
+            const bool need = m_tile > m_ref + kTau;
+            if (__any_sync(0xffffffffu, need)) {
+                const float m_new = need ? m_tile : m_ref;
+                const float alpha = (m_ref == neg_inf()) ? 0.f : ex2_approx(m_ref - m_new);
+                l *= alpha;
+                if (j > 0) {
+                    // O_i row *= alpha (O is stable: the MMA that produced this
+                    // S tile was issued after the previous P.V and its commit
+                    // covers it).
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orr[32];
+                        tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32dp_x32(tO + cc * 32, orr);
+                    }
+                }
+                m_ref = m_new;
+            }
+            const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
+            uint32_t pk[64];
+            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; c += 2) {
+                float p0, p1;
+                if constexpr (HAS_BIAS) {
+                    p0 = ex2_approx(x[c] - m_use);
+                    p1 = ex2_approx(x[c + 1] - m_use);
+                } else {
+                    p0 = ex2_approx(fmaf(x[c], qk, -m_use));
+                    p1 = ex2_approx(fmaf(x[c + 1], qk, -m_use));
+                }
+                l0 += p0;
+                l1 += p1;
+                pk[c >> 1] = pack2<BF16>(p0, p1);
+            }
+            l += l0 + l1;
+            tmem_st32dp_x64(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::kPFull + i));
+        }
+
+        // ---- epilogue: O = o / l, LSE = (m_ref + log2 l) ln 2
+        if (ok && n_kv > 0) {
+            const bool got = mbar_wait(bar(L::kOFull + i), 0, wctx);
+            ok = __all_sync(0xffffffffu, got);
+            tc_fence_after();
+        }
+        if (ok) {
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            uint8_t *stage = smem + L::kQ + i * L::kTileBytes;   // Q_i is dead now
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t orr[32];
+                if (n_kv > 0) {
+                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
+                                        __uint_as_float(orr[2 * e + 1]) * inv_l);
+                // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
+                const int chunk = (cc * 32) / 64;
+                const int k16_base = ((cc * 32) % 64) / 8;
+                uint8_t *rowp = stage + chunk * L::kChunkBytes + row * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int k16 = (k16_base + q4) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(rowp + k16 * 16) =
+                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+            if (qrow < p.Nq) {
+                const float lse = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : neg_inf();
+                p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = lse;
+            }
+            // each warp stores its own 32 rows (box 64 x 32)
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int row0 = m0 + i * kBM + wq * 32;
+            if (lane == 0 && row0 < p.Nq) {
+                for (int c = 0; c < D / 64; ++c)
+                    tma_store_3d(&tm_o, sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes + wq * 32 * 128,
+                                 c * 64, row0, bh);
+                tma_store_commit();
+                tma_store_wait_all();
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+// Rows with no key at all (Nk == 0): O = 0, LSE = -inf.
+template <typename T>
+__global__ void fa_fwd_empty_kernel(T *o, float *lse, size_t n_rows, int D) {
+    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+    for (size_t r = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; r < n_rows; r += stride) {
+        lse[r] = __int_as_float(0xff800000);
+        for (int d = 0; d < D; ++d) o[r * D + d] = T(0.f);
+    }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, cudaStream_t stream) {
+    using L = FwdLayout<D>;
+    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H;
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_fwd_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias,
+                         cudaStream_t s) {
+    if (causal) return bias ? launch_fwd_t<D, BF16, true, true>(tm, p, s) : launch_fwd_t<D, BF16, true, false>(tm, p, s);
+    return bias ? launch_fwd_t<D, BF16, false, true>(tm, p, s) : launch_fwd_t<D, BF16, false, false>(tm, p, s);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                       bool has_bias, cudaStream_t stream) {
+    if (D == 64) return bf16 ? launch_fwd_d<64, true>(tm, p, causal, has_bias, stream)
+                             : launch_fwd_d<64, false>(tm, p, causal, has_bias, stream);
+    return bf16 ? launch_fwd_d<128, true>(tm, p, causal, has_bias, stream)
+                : launch_fwd_d<128, false>(tm, p, causal, has_bias, stream);
+}
+
+cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16, cudaStream_t stream) {
+    const unsigned grid = static_cast<unsigned>(std::min<size_t>((n_rows + 255) / 256, 4096));
+    if (grid == 0) return cudaSuccess;
+    if (bf16)
+        fa_fwd_empty_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(o), lse, n_rows, D);
+    else
+        fa_fwd_empty_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<__half *>(o), lse, n_rows, D);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,33 @@
+// fa_internal.h -- structures shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace fa {
+
+// Forward launch parameters (everything except the tensor maps).
+struct FwdParams {
+    int B, H, Nq, Nk;
+    int n_mblocks;                 // ceil(Nq / 256): work units per (b, h)
+    int causal_off;                // Nk - Nq (bottom-right causal alignment)
+    float qk_scale_log2;           // scale * log2(e)
+    const float *bias;             // [B, Nk] or nullptr
+    float *lse;                    // [B*H, Nq]
+    int *err;                      // device error word
+    unsigned long long timeout_ns; // limit of every device-side wait
+};
+
+struct FwdTensorMaps {
+    CUtensorMap q, k, v, o;
+};
+
+cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                       bool has_bias, cudaStream_t stream);
+cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,
+                             cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,122 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * The operation is exact scaled dot-product attention
+ *
+ *     O = softmax(scale * Q K^T + mask) V
+ *
+ * as defined on the FlashAttention case-study slides (nmj0.github.io,
+ * "Attention is where tokens meet"), computed as on the slide "FlashAttention:
+ * the idea": one fused, tiled kernel that never writes the score matrix S or
+ * the probability matrix P to device memory, combining key tiles with the
+ * running (m, l, o) update of "Online softmax: divide once, at the end" and
+ * dividing by l once per row.  The backward pass recomputes the scores from
+ * the saved row log-sum-exp instead of storing them (lastdictionary.com,
+ * "FlashAttention", definition paragraph).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers    Every tensor pointer is DEVICE memory owned by the caller and
+ *             must be 16-byte aligned.  The library keeps no pointer after a
+ *             call returns and allocates no device memory per call (the
+ *             backward's scratch comes from the caller's `workspace`).
+ * Layout      q, o, dO, dq: [B, H, Nq, D]; k, v, dk, dv: [B, H, Nk, D];
+ *             contiguous, row-major, D fastest (the "reshape to [h x n x d_k]"
+ *             of the slides' "Queries, keys and values").  All share `dtype`.
+ *             lse: [B, H, Nq] float32.  key_bias: [B, Nk] float32.
+ * dtype       FA_F16 or FA_BF16 (storage and tensor-core input type; all
+ *             accumulation is float32).
+ * D           64 or 128.
+ * Sizes       B, H >= 1; Nq, Nk >= 0.  Nq == 0 is a no-op (no pointer is
+ *             read).  Nk == 0 makes every row empty (O = 0, LSE = -inf);
+ *             k, v (and dk, dv) may then be NULL.
+ * scale       Multiplies Q K^T before the mask; finite and > 0 (pass
+ *             1/sqrt(D) for standard attention).
+ * causal      0 or 1.  Bottom-right aligned: key j is visible to query i iff
+ *             j <= i + (Nk - Nq), which is j <= i when Nq == Nk.
+ * key_bias    Optional (NULL = none).  Additive per-key term added to the
+ *             scaled scores of batch b, shared by all heads and queries;
+ *             entries are finite or -inf (-inf = masked key).
+ * Empty rows  A query row that sees no key gets O = 0 and LSE = -inf.
+ * stream      A cudaStream_t passed as void*; NULL = the legacy default
+ *             stream.  Work is enqueued asynchronously on it.
+ * Errors      Argument errors are reported synchronously, before anything is
+ *             launched.  Kernel launch failures return FA_ERR_CUDA.  A device
+ *             wait that exceeds its time limit makes the kernel give up
+ *             cleanly and latch FA_ERR_DEVICE_TIMEOUT in a per-device error
+ *             word, read and cleared by fa_device_status().
+ * Threads     Calls on different streams may run concurrently.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size, bad scale */
+    FA_ERR_UNSUPPORTED = 2,     /* D not in {64, 128}, unknown dtype, no sm_100 device */
+    FA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
+    FA_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device-side wait gave up */
+    FA_ERR_WORKSPACE = 5        /* backward workspace missing or too small */
+} fa_status;
+
+typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/*
+ * Forward pass.  Writes o [B,H,Nq,D] (dtype) and lse [B,H,Nq] (float32,
+ * natural log of sum_j exp(scale * q_i . k_j + bias_j) over visible keys).
+ * Inputs are read once per query tile from HBM; S and P live only on chip.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int Nq, int Nk, int D, int causal, float scale,
+           int dtype, const float *key_bias, void *stream);
+
+/*
+ * Bytes of device scratch fa_bwd() needs for these sizes: the per-row term
+ * D_i = rowsum(dO * O) (float32) and a float32 dQ accumulator.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D);
+
+/*
+ * Backward pass of L = sum(O * dO): writes dq, dk, dv (dtype, same layouts as
+ * q, k, v).  o and lse must be the outputs of fa_fwd() for the same inputs.
+ * Scores and probabilities are recomputed tile by tile from q, k and lse.
+ * workspace: device memory of at least fa_bwd_workspace_bytes() bytes,
+ * 16-byte aligned, owned by the caller; its contents on entry do not matter.
+ * The mask and key_bias receive no gradient.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o,
+           const float *lse, const void *dO, void *dq, void *dk, void *dv,
+           int B, int H, int Nq, int Nk, int D, int causal, float scale,
+           int dtype, const float *key_bias, void *workspace,
+           size_t workspace_bytes, void *stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error
+ * word: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait since
+ * the last call.  FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_device_status(void *stream);
+
+/*
+ * Self-test of the bounded-wait mechanism: launches one block that waits on a
+ * barrier nothing will ever complete, with a limit of `timeout_us`
+ * microseconds; the kernel must give up, latch FA_ERR_DEVICE_TIMEOUT and
+ * return.  Returns FA_OK if the launch succeeded (read the outcome with
+ * fa_device_status()).
+ */
+int fa_debug_wait_timeout(unsigned timeout_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/fa.h declares, and rejects bad arguments synchronously (before any
+CUDA call) with the documented status codes."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import exact_attention_112_b200 as fa
+from exact_attention_112_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return fa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string",
+            "fa_device_status"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r" T (\w+)$", out, flags=re.M))
+    for n in names:
+        assert n in exported, f"{n} declared in fa.h but not exported"
+        assert hasattr(L, n)
+
+
+def test_status_strings(L):
+    for code in range(6):
+        s = fa.fa_status_string(code)
+        assert s and s.startswith("FA_")
+    assert "unknown" in fa.fa_status_string(99)
+
+
+def _fwd(L, q=1, k=1, v=1, o=1, lse=1, B=1, H=1, Nq=128, Nk=128, D=64, causal=0,
+         scale=0.125, dtype=0, bias=None):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    return L.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, Nq, Nk, D, causal,
+                    ctypes.c_float(scale), dtype, P(bias), None)
+
+
+def test_fwd_argument_errors_are_synchronous(L):
+    assert _fwd(L, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, D=256) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, dtype=7) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, B=0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, H=-1) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, Nk=-3) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, causal=2) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=0.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, q=0) == fa.FA_ERR_INVALID_ARG          # null pointer
+    assert _fwd(L, lse=0) == fa.FA_ERR_INVALID_ARG
+    # misaligned (not a multiple of 16 bytes)
+    assert L.fa_fwd(ctypes.c_void_p(24), ctypes.c_void_p(32), ctypes.c_void_p(48),
+                    ctypes.c_void_p(64), ctypes.c_void_p(80), 1, 1, 128, 128, 64, 0,
+                    ctypes.c_float(0.1), 0, None, None) == fa.FA_ERR_INVALID_ARG
+    # index overflow guard
+    assert _fwd(L, B=1 << 16, H=1 << 16) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fwd_empty_query_is_a_noop(L):
+    # Nq == 0: nothing to compute, no CUDA call, even with null pointers
+    assert _fwd(L, q=None, k=None, v=None, o=None, lse=None, Nq=0) == fa.FA_OK
+
+
+def test_workspace_size(L):
+    B, H, N, D = 2, 32, 4096, 128
+    ws = fa.fa_bwd_workspace_bytes(B, H, N, N, D)
+    rows = B * H * N
+    assert ws >= rows * 4 + rows * D * 4
+    assert ws < rows * 4 + rows * D * 4 + 4096
+    assert fa.fa_bwd_workspace_bytes(1, 1, 256, 256, 96) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(fa, "_lib", None)
+    monkeypatch.setattr(fa, "library_path", lambda: str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        fa.lib()
