@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the fused exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama] [--dtype bf16] [--passes fwd,bwd]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the forward (and, with the backward built, the backward) of one Llama-3-8B
+attention layer, B=1, H=32, Nq=Nk=8192, d_k=128, causal (the shapes of the
+FlashAttention case-study slides, "The same computation at real size").
+
+value    = algorithmic TFLOP/s of the step (4*B*H*Nq*Nk*D forward, halved for
+           causal; 2.5x that for the backward), inputs resident in HBM, L2
+           flushed between steps, timed with CUDA events on the launch stream.
+e2e      = the same metric through the public binding with HOST buffers:
+           pinned-host -> device copies of the step's inputs and the device ->
+           host read of its outputs are inside the timed region.
+roofline = the dominant kernel's achieved TFLOP/s against the measured bf16
+           tensor-core peak (MEASURED_PEAKS.json).
+cpu_baseline = the float64 oracle on a bounded row sample, on host cores.
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
+GPU (independent (batch, head) shards, no collective on the data path): weak
+scaling; value = all ranks' FLOPs / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and fraction of dense BF16/FP16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"])
+    ap.add_argument("--passes", default="fwd", help="comma list of fwd,bwd")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target oracle CPU time of the cpu_baseline sample")
+    ap.add_argument("--flush-mib", type=int, default=512)
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_cfg(args):
+    from exact_attention_112_b200 import inputs
+    w = inputs.workload(args.workload, dtype=args.dtype)
+    return w
+
+
+def flops_of(w, passes):
+    from exact_attention_112_b200 import metrics
+    f = {}
+    if "fwd" in passes:
+        f["fwd"] = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    if "bwd" in passes:
+        f["bwd"] = metrics.bwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    return f
+
+
+def workload_name(w, passes):
+    return (f"llama-3-8b layer attention {'+'.join(passes)}: B={w['B']} H={w['H']} "
+            f"Nq={w['Nq']} Nk={w['Nk']} D={w['D']} "
+            f"{'causal' if w['causal'] else 'non-causal'} {w['dtype']}")
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        self.dev = device_index
+
+    def start(self):
+        import tempfile
+        self.path = tempfile.mktemp(suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3])
+                          if v.lower().startswith("active")})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample_setup(w):
+    """Host float64 inputs of the workload for the oracle."""
+    from exact_attention_112_b200 import inputs
+    inp = inputs.make_inputs(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], dtype=w["dtype"],
+                             seed=w["seed"], qk_std=w["qk_std"], v_dist=w["v_dist"],
+                             bias_frac=w["bias_frac"])
+    f = inputs.to_f64
+    return {k: f(inp[k]) for k in ("q", "k", "v", "key_bias")}
+
+
+def oracle_rows_time(arrs, w, rows):
+    """Run the oracle forward on `rows` of every (b, h); return (seconds,
+    algorithmic FLOPs of those rows)."""
+    import numpy as np
+    import oracle
+    t0 = time.perf_counter()
+    oracle.fwd(arrs["q"], arrs["k"], arrs["v"], arrs["key_bias"], w["causal"],
+               1.0 / math.sqrt(w["D"]), rows=rows)
+    dt = time.perf_counter() - t0
+    rows = np.asarray(rows)
+    if w["causal"]:
+        vis = np.clip(rows + (w["Nk"] - w["Nq"]) + 1, 0, w["Nk"])
+    else:
+        vis = np.full(rows.shape, w["Nk"])
+    fl = 4.0 * w["D"] * float(vis.sum()) * w["B"] * w["H"]
+    return dt, fl
+
+
+def pick_rows(w, n):
+    import numpy as np
+    return np.unique(np.linspace(0, w["Nq"] - 1, max(1, n)).round().astype(np.int64))
+
+
+def cpu_baseline(w, target_s):
+    import oracle
+    arrs = oracle_sample_setup(w)
+    cores = oracle.max_threads()
+    dt, fl = oracle_rows_time(arrs, w, pick_rows(w, 4))          # calibration
+    n = max(4, int(4 * target_s / max(dt, 1e-3)))
+    rows = pick_rows(w, min(n, w["Nq"]))
+    dt, fl = oracle_rows_time(arrs, w, rows)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"float64 oracle forward on {len(rows)} evenly spaced query rows of "
+                       f"each of the {w['B'] * w['H']} (b,h) pairs ({fl / 1e9:.1f} GFLOP "
+                       f"algorithmic, {dt:.1f} s)"),
+            "seconds": dt}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded row sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = workload_cfg(args)
+    passes = [p for p in args.passes.split(",") if p]
+    arrs = oracle_sample_setup(w)
+    cores = oracle.max_threads()
+    dt, _ = oracle_rows_time(arrs, w, pick_rows(w, 2))
+    budget = 150.0 / max(1, args.steps + args.warmup)   # whole run within a few minutes
+    n = max(1, int(2 * budget / max(dt, 1e-4)))
+    rows = pick_rows(w, min(n, w["Nq"]))
+    for _ in range(args.warmup):
+        oracle_rows_time(arrs, w, rows)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_rows_time(arrs, w, rows)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(w, passes), "B": w["B"], "H": w["H"],
+                   "Nq": w["Nq"], "Nk": w["Nk"], "D": w["D"], "causal": w["causal"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": (f"each step: float64 oracle forward on {len(rows)} "
+                                    f"evenly spaced query rows of all {w['B'] * w['H']} "
+                                    "(b,h) pairs")},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_112_b200 as fa
+    from exact_attention_112_b200 import inputs, metrics
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    passes = [p for p in args.passes.split(",") if p]
+    w = workload_cfg(args)
+    B, H, Nq, Nk, D, causal = w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"]
+    # every rank draws its own (b, h) shard of a larger batch: seed by rank
+    inp = inputs.make_inputs(B, H, Nq, Nk, D, dtype=w["dtype"], seed=w["seed"] + 7 * rank,
+                             qk_std=w["qk_std"], v_dist=w["v_dist"], bias_frac=w["bias_frac"],
+                             with_dO="bwd" in passes)
+    q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+    bias = None if inp["key_bias"] is None else inp["key_bias"].to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    if "bwd" in passes:
+        dO = inp["do"].to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(fa.fa_bwd_workspace_bytes(B, H, Nq, Nk, D), dtype=torch.uint8, device=dev)
+    flush = torch.empty(args.flush_mib * (1 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_fwd(q, k, v, o, lse, causal=causal, key_bias=bias, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if "bwd" in passes:
+            fa.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, causal=causal, key_bias=bias,
+                      stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    assert fa.fa_device_status(stream) == fa.FA_OK
+
+    n_ev = 3 if "bwd" in passes else 2
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = fa.fa_launch_count()
+    for s in range(args.steps):
+        flush.zero_()                      # L2 flush outside the timed events
+        step(evs[s])
+    torch.cuda.synchronize(dev)
+    launches = fa.fa_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    st = fa.fa_device_status(stream)
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status after timing: {fa.fa_status_string(st)}")
+
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if "bwd" in passes else []
+    step_ms = [f + b for f, b in zip(fwd_ms, bwd_ms or [0.0] * len(fwd_ms))]
+    t_local = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([t_local], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    else:
+        t_max = t_local
+    fl = flops_of(w, passes)
+    step_flops = sum(fl.values())
+    value = world * step_flops * args.steps / (t_max * 1e-3) / 1e12
+
+    # ---- end to end through the public binding, host buffers
+    host = {x: inp[x].pin_memory() for x in ("q", "k", "v")}
+    if "bwd" in passes:
+        host["do"] = inp["do"].pin_memory()
+    out_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    out_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    outs_b = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in (q, k, v)] \
+        if "bwd" in passes else []
+    h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
+    d2h = out_o.numel() * out_o.element_size() + out_lse.numel() * 4 + \
+        sum(t_.numel() * t_.element_size() for t_ in outs_b)
+
+    def e2e_step():
+        q.copy_(host["q"], non_blocking=True)
+        k.copy_(host["k"], non_blocking=True)
+        v.copy_(host["v"], non_blocking=True)
+        fa.fa_fwd(q, k, v, o, lse, causal=causal, key_bias=bias, stream=stream)
+        out_o.copy_(o, non_blocking=True)
+        out_lse.copy_(lse, non_blocking=True)
+        if "bwd" in passes:
+            dO.copy_(host["do"], non_blocking=True)
+            fa.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, causal=causal, key_bias=bias,
+                      stream=stream)
+            for dst, src in zip(outs_b, (dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * step_flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    kern_ms = {"fwd": statistics.mean(fwd_ms)}
+    if bwd_ms:
+        kern_ms["bwd"] = statistics.mean(bwd_ms)
+    dom = max(kern_ms, key=kern_ms.get)
+    peak = float(peaks["bf16_tflops"])
+    achieved = fl[dom] / (kern_ms[dom] * 1e-3) / 1e12
+    traffic = load_traffic(dom, w)
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+            "frac": achieved / peak, "traffic": traffic, "kernel": f"fa_{dom}",
+            "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+            else "fallback 1.59 PFLOP/s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+        "config": {"workload": workload_name(w, passes), "B": B, "H": H, "Nq": Nq, "Nk": Nk,
+                   "D": D, "causal": causal, "passes": passes,
+                   "l2": f"flushed between steps ({args.flush_mib} MiB write, outside the events)",
+                   "parallelism": "replicas" if world == 1 else f"{world} ranks, independent (b,h) shards"},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "per_pass": {p: {"ms": kern_ms[p], "tflops": fl[p] / (kern_ms[p] * 1e-3) / 1e12,
+                         "frac_of_peak": fl[p] / (kern_ms[p] * 1e-3) / 1e12 / peak}
+                     for p in kern_ms},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(kind, w):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/), or None if none matches the current kernel build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        d = json.load(open(path))
+        ent = d.get(f"fa_{kind}:{w['name']}")
+        if ent and ent.get("kernel_rev") == kernel_rev():
+            return ent["bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def kernel_rev():
+    """Content hash of the CUDA sources, so stale ncu traffic is not reported."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "exact_attention_112_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

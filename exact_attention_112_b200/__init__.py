@@ -23,7 +23,7 @@ __all__ = [
     "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_F16", "FA_BF16", "FaError",
     "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes",
-    "fa_status_string", "fa_device_status", "fa_debug_wait_timeout",
+    "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "attention_forward", "attention_backward",
 ]
 
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
             L.fa_status_string.restype = ctypes.c_char_p
             L.fa_device_status.argtypes = [vp]
             L.fa_device_status.restype = i
+            L.fa_launch_count.argtypes = []
+            L.fa_launch_count.restype = ctypes.c_ulonglong
             L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
             L.fa_debug_wait_timeout.restype = i
             _lib = L
@@ -141,6 +143,10 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, causal=False, scale=None,
 
 def fa_device_status(stream=None) -> int:
     return int(lib().fa_device_status(_stream_ptr(stream)))
+
+
+def fa_launch_count() -> int:
+    return int(lib().fa_launch_count())
 
 
 def fa_debug_wait_timeout(timeout_us: int, stream=None) -> int:

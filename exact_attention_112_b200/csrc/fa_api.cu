@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -101,9 +102,15 @@ int check_common(int B, int H, int Nq, int Nk, int D, int causal, float scale, i
     return FA_OK;
 }
 
+std::atomic<unsigned long long> g_launches{0};
+
 }  // namespace
 
+void fa::note_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
 extern "C" {
+
+unsigned long long fa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *fa_status_string(int status) {
     switch (status) {
@@ -219,5 +226,6 @@ extern "C" int fa_debug_wait_timeout(unsigned timeout_us, void *stream) {
     if (timeout_us == 0 || timeout_us > 10000000u) return FA_ERR_INVALID_ARG;
     fa_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         err, static_cast<unsigned long long>(timeout_us) * 1000ull);
+    fa::note_launch();
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -473,6 +473,7 @@ cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, cudaStream
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H;
     kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -500,6 +501,7 @@ cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf1
         fa_fwd_empty_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(o), lse, n_rows, D);
     else
         fa_fwd_empty_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<__half *>(o), lse, n_rows, D);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -25,6 +25,9 @@ struct FwdTensorMaps {
     CUtensorMap q, k, v, o;
 };
 
+// Counts every kernel launch made by the library (fa_launch_count()).
+void note_launch(unsigned n = 1);
+
 cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                        bool has_bias, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,

@@ -107,6 +107,12 @@ const char *fa_status_string(int status);
 int fa_device_status(void *stream);
 
 /*
+ * Number of kernels this library has launched in this process (all devices,
+ * all streams) since it was loaded; for accounting in benchmarks.
+ */
+unsigned long long fa_launch_count(void);
+
+/*
  * Self-test of the bounded-wait mechanism: launches one block that waits on a
  * barrier nothing will ever complete, with a limit of `timeout_us`
  * microseconds; the kernel must give up, latch FA_ERR_DEVICE_TIMEOUT and
