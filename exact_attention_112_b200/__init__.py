@@ -21,13 +21,14 @@ import threading
 
 __all__ = [
     "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
-    "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_F16", "FA_BF16", "FaError",
+    "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
     "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "attention_forward", "attention_backward",
 ]
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+(FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT,
+ FA_ERR_WORKSPACE, FA_ERR_INTERNAL) = range(7)
 FA_F16, FA_BF16 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

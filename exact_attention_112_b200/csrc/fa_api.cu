@@ -120,6 +120,7 @@ const char *fa_status_string(int status) {
         case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
         case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a device-side wait gave up";
         case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: backward workspace missing or too small";
+        case FA_ERR_INTERNAL: return "FA_ERR_INTERNAL: a kernel's layout self-check failed";
         default: return "unknown fa_status";
     }
 }
@@ -177,10 +178,61 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
            int causal, float scale, int dtype, const float *key_bias, void *workspace,
            size_t workspace_bytes, void *stream) {
-    (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dO; (void)dq; (void)dk; (void)dv;
-    (void)B; (void)H; (void)Nq; (void)Nk; (void)D; (void)causal; (void)scale; (void)dtype;
-    (void)key_bias; (void)workspace; (void)workspace_bytes; (void)stream;
-    return FA_ERR_UNSUPPORTED;
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (Nq > 0 && (!q || !o || !lse || !dO || !dq)) return FA_ERR_INVALID_ARG;
+    if (Nk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, key_bias, workspace};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+    const size_t need = fa_bwd_workspace_bytes(B, H, Nq, Nk, D);
+    if (Nq > 0 && (!workspace || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    const long long BH = static_cast<long long>(B) * H;
+    if (Nq == 0) {
+        // no query: every key and value gradient is zero
+        if (Nk == 0) return FA_OK;
+        const size_t bytes = static_cast<size_t>(BH) * Nk * D * 2;
+        if (cudaMemsetAsync(dk, 0, bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, s) != cudaSuccess)
+            return FA_ERR_CUDA;
+        return FA_OK;
+    }
+    const size_t rows = static_cast<size_t>(BH) * Nq;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    fa::BwdParams p;
+    p.B = B;
+    p.H = H;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.causal_off = Nk - Nq;
+    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    p.scale = scale;
+    p.bias = key_bias;
+    p.lse = lse;
+    p.o = o;
+    p.dO = dO;
+    p.Di = static_cast<float *>(workspace);
+    p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + up(rows * sizeof(float)));
+    p.dq = dq;
+    p.err = err;
+    p.timeout_ns = kDefaultTimeoutNs;
+    fa::BwdTensorMaps tm;
+    std::memset(&tm, 0, sizeof(tm));
+    if (Nk > 0) {
+        if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.dO, dO, bf16, D, Nq, BH, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.dk, dk, bf16, D, Nk, BH, 32)) != FA_OK) return st;
+        if ((st = make_map(&tm.dv, dv, bf16, D, Nk, BH, 32)) != FA_OK) return st;
+    }
+    cudaError_t e = fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_device_status(void *stream) {

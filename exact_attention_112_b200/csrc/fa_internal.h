@@ -25,6 +25,29 @@ struct FwdTensorMaps {
     CUtensorMap q, k, v, o;
 };
 
+// Backward launch parameters.
+struct BwdParams {
+    int B, H, Nq, Nk;
+    int causal_off;                // Nk - Nq
+    float qk_scale_log2;           // scale * log2(e)
+    float scale;
+    const float *bias;             // [B, Nk] or nullptr
+    const float *lse;              // [B*H, Nq] from the forward
+    const void *o, *dO;            // [B*H, Nq, D] 16-bit
+    float *Di;                     // workspace: [B*H*Nq]
+    float *dq_acc;                 // workspace: [B*H*Nq, D] fp32
+    void *dq;                      // [B*H, Nq, D] 16-bit output
+    int *err;
+    unsigned long long timeout_ns;
+};
+
+struct BwdTensorMaps {
+    CUtensorMap q, k, v, dO, dk, dv;
+};
+
+cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
+                       bool has_bias, cudaStream_t stream);
+
 // Counts every kernel launch made by the library (fa_launch_count()).
 void note_launch(unsigned n = 1);
 

@@ -14,6 +14,7 @@ namespace fa {
 
 // Device error codes latched by the kernels (same values as fa_status).
 constexpr int kErrDeviceTimeout = 4;
+constexpr int kErrInternal = 6;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

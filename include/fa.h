@@ -62,7 +62,8 @@ typedef enum {
     FA_ERR_UNSUPPORTED = 2,     /* D not in {64, 128}, unknown dtype, no sm_100 device */
     FA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
     FA_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device-side wait gave up */
-    FA_ERR_WORKSPACE = 5        /* backward workspace missing or too small */
+    FA_ERR_WORKSPACE = 5,       /* backward workspace missing or too small */
+    FA_ERR_INTERNAL = 6         /* a kernel's own layout check failed; it did no work */
 } fa_status;
 
 typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
