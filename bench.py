@@ -85,8 +85,13 @@ def flops_of(w, passes):
     return f
 
 
+WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention backward workload",
+                   "tiny": "tiny attention", "stress": "numerical-stress attention",
+                   "sweep": "sequence-sweep attention"}
+
+
 def workload_name(w, passes):
-    return (f"llama-3-8b layer attention {'+'.join(passes)}: B={w['B']} H={w['H']} "
+    return (f"{WORKLOAD_TITLES.get(w['name'], w['name'])} {'+'.join(passes)}: B={w['B']} H={w['H']} "
             f"Nq={w['Nq']} Nk={w['Nk']} D={w['D']} "
             f"{'causal' if w['causal'] else 'non-causal'} {w['dtype']}")
 
@@ -150,31 +155,37 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle sample (cpu_baseline and the reference arm)
 # --------------------------------------------------------------------------
-def oracle_sample_setup(w):
+def oracle_sample_setup(w, passes):
     """Host float64 inputs of the workload for the oracle."""
     from exact_attention_112_b200 import inputs
     inp = inputs.make_inputs(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], dtype=w["dtype"],
                              seed=w["seed"], qk_std=w["qk_std"], v_dist=w["v_dist"],
-                             bias_frac=w["bias_frac"])
+                             bias_frac=w["bias_frac"], with_dO="bwd" in passes)
     f = inputs.to_f64
-    return {k: f(inp[k]) for k in ("q", "k", "v", "key_bias")}
+    return {k: f(inp[k]) for k in ("q", "k", "v", "key_bias", "do")}
 
 
-def oracle_rows_time(arrs, w, rows):
-    """Run the oracle forward on `rows` of every (b, h); return (seconds,
-    algorithmic FLOPs of those rows)."""
+def oracle_rows_time(arrs, w, rows, passes):
+    """Run the oracle's passes on the query rows `rows` of every (b, h); return
+    (seconds, algorithmic FLOPs of that share of the step)."""
     import numpy as np
     import oracle
+    scale = 1.0 / math.sqrt(w["D"])
     t0 = time.perf_counter()
-    oracle.fwd(arrs["q"], arrs["k"], arrs["v"], arrs["key_bias"], w["causal"],
-               1.0 / math.sqrt(w["D"]), rows=rows)
+    if "fwd" in passes:
+        oracle.fwd(arrs["q"], arrs["k"], arrs["v"], arrs["key_bias"], w["causal"], scale,
+                   rows=rows)
+    if "bwd" in passes:
+        oracle.bwd(arrs["q"], arrs["k"], arrs["v"], arrs["do"], arrs["key_bias"], w["causal"],
+                   scale, rows=rows)
     dt = time.perf_counter() - t0
     rows = np.asarray(rows)
     if w["causal"]:
         vis = np.clip(rows + (w["Nk"] - w["Nq"]) + 1, 0, w["Nk"])
     else:
         vis = np.full(rows.shape, w["Nk"])
-    fl = 4.0 * w["D"] * float(vis.sum()) * w["B"] * w["H"]
+    per_fwd = 4.0 * w["D"] * float(vis.sum()) * w["B"] * w["H"]
+    fl = (per_fwd if "fwd" in passes else 0.0) + (2.5 * per_fwd if "bwd" in passes else 0.0)
     return dt, fl
 
 
@@ -183,18 +194,21 @@ def pick_rows(w, n):
     return np.unique(np.linspace(0, w["Nq"] - 1, max(1, n)).round().astype(np.int64))
 
 
-def cpu_baseline(w, target_s):
+def sample_text(w, rows, passes):
+    return (f"float64 oracle {'+'.join(passes)} on {len(rows)} evenly spaced query rows of "
+            f"each of the {w['B'] * w['H']} (b,h) pairs")
+
+
+def cpu_baseline(w, target_s, passes):
     import oracle
-    arrs = oracle_sample_setup(w)
+    arrs = oracle_sample_setup(w, passes)
     cores = oracle.max_threads()
-    dt, fl = oracle_rows_time(arrs, w, pick_rows(w, 4))          # calibration
-    n = max(4, int(4 * target_s / max(dt, 1e-3)))
+    dt, fl = oracle_rows_time(arrs, w, pick_rows(w, 8), passes)          # calibration
+    n = max(8, int(8 * target_s / max(dt, 1e-3)))
     rows = pick_rows(w, min(n, w["Nq"]))
-    dt, fl = oracle_rows_time(arrs, w, rows)
+    dt, fl = oracle_rows_time(arrs, w, rows, passes)
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": (f"float64 oracle forward on {len(rows)} evenly spaced query rows of "
-                       f"each of the {w['B'] * w['H']} (b,h) pairs ({fl / 1e9:.1f} GFLOP "
-                       f"algorithmic, {dt:.1f} s)"),
+            "sample": sample_text(w, rows, passes) + f" ({fl / 1e9:.1f} GFLOP algorithmic, {dt:.1f} s)",
             "seconds": dt}
 
 
@@ -206,17 +220,17 @@ def run_reference(args):
     import oracle
     w = workload_cfg(args)
     passes = [p for p in args.passes.split(",") if p]
-    arrs = oracle_sample_setup(w)
+    arrs = oracle_sample_setup(w, passes)
     cores = oracle.max_threads()
-    dt, _ = oracle_rows_time(arrs, w, pick_rows(w, 2))
+    dt, _ = oracle_rows_time(arrs, w, pick_rows(w, 4), passes)
     budget = 150.0 / max(1, args.steps + args.warmup)   # whole run within a few minutes
-    n = max(1, int(2 * budget / max(dt, 1e-4)))
+    n = max(2, int(4 * budget / max(dt, 1e-4)))
     rows = pick_rows(w, min(n, w["Nq"]))
     for _ in range(args.warmup):
-        oracle_rows_time(arrs, w, rows)
+        oracle_rows_time(arrs, w, rows, passes)
     tot_t, tot_f = 0.0, 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_rows_time(arrs, w, rows)
+        dt, fl = oracle_rows_time(arrs, w, rows, passes)
         tot_t += dt
         tot_f += fl
     value = tot_f / tot_t / 1e12
@@ -226,11 +240,10 @@ def run_reference(args):
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(w, passes), "B": w["B"], "H": w["H"],
-                   "Nq": w["Nq"], "Nk": w["Nk"], "D": w["D"], "causal": w["causal"]},
+                   "Nq": w["Nq"], "Nk": w["Nk"], "D": w["D"], "causal": w["causal"],
+                   "passes": passes},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": (f"each step: float64 oracle forward on {len(rows)} "
-                                    f"evenly spaced query rows of all {w['B'] * w['H']} "
-                                    "(b,h) pairs")},
+                         "sample": "each step: " + sample_text(w, rows, passes)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -402,7 +415,7 @@ def run_ours(args):
                      for p in kern_ms},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, passes)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -85,6 +85,23 @@ int make_map(CUtensorMap *m, const void *ptr, bool bf16, int D, int N, long long
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// 3-D fp32 map over the [B*H, Nq, D] dQ accumulator: 32 x 32 boxes with the
+// 128-byte swizzle, used by the TMA reduce-add of dQ contributions.
+int make_map_f32(CUtensorMap *m, void *ptr, int D, int N, long long BH) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int st = get_encoder(&enc);
+    if (st != FA_OK) return st;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(N) * D * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shared shape/scalar validation of forward and backward.
@@ -230,6 +247,7 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
         if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
         if ((st = make_map(&tm.dk, dk, bf16, D, Nk, BH, 32)) != FA_OK) return st;
         if ((st = make_map(&tm.dv, dv, bf16, D, Nk, BH, 32)) != FA_OK) return st;
+        if ((st = make_map_f32(&tm.dqacc, p.dq_acc, D, Nq, BH)) != FA_OK) return st;
     }
     cudaError_t e = fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -22,14 +22,14 @@
 //        dV  += P^T dO_j   (P^T from tensor memory)
 //        dK  += dS^T Q_j   (dS^T from shared memory, K-major)
 //        dQ_j = dS K       (the same dS^T buffer read as an MN-major operand)
-//      and a readout warpgroup adds scale * dQ_j into dQacc with vector
-//      atomics.  dK (x scale) and dV are written once at the end.
+//      and a readout warpgroup adds scale * dQ_j into dQacc with TMA bulk
+//      reduce-add (fp32).  dK (x scale) and dV are written once at the end.
 //   3. fa_bwd_dq_convert_kernel  dQ = dQacc cast to the 16-bit type.
 //
 // Tensor memory of the dK/dV kernel (lane = key row, except dQ: lane = query):
 //   cols [0,128)      S^T (fp32); P^T (16-bit pairs) overwrites cols [0,64)
-//   cols [128,256)    dP^T (fp32)
-//   cols [64,64+D)    dQ_j (fp32), written after S^T and dP^T have been read
+//   cols [128,256)    dP^T (fp32); dQ_j (fp32) in cols [128,128+D) once dS^T
+//                     has been formed from it
 //   cols [256,256+D)  dV accumulator,  cols [256+D,256+2D) dK accumulator
 // Warp roles (10 warps): 0-3 recompute/gradient, 4-7 dQ readout, 8 TMA
 // producer (also stages LSE and D of each query tile), 9 MMA issuer.
@@ -70,16 +70,18 @@ struct BwdLayout {
     static constexpr int kQFull = 1;    // +stage
     static constexpr int kQEmpty = 3;   // +stage
     static constexpr int kSFull = 5;
-    static constexpr int kPFull = 6;
-    static constexpr int kDQFull = 7;
-    static constexpr int kDQEmpty = 8;
-    static constexpr int kAccFull = 9;
-    static constexpr int kDrain = 10;
-    static constexpr int kNumBars = 11;
+    static constexpr int kPTFull = 6;
+    static constexpr int kDPFull = 7;
+    static constexpr int kDSFull = 8;
+    static constexpr int kDQFull = 9;
+    static constexpr int kDQEmpty = 10;
+    static constexpr int kAccFull = 11;
+    static constexpr int kDrain = 12;
+    static constexpr int kNumBars = 13;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 64, kColDV = 256, kColDK = 256 + D;
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -160,13 +162,21 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float4 *__
 
 // ---------------------------------------------------------------------------
 // 2. dK, dV (and dQ contributions) for one 128-key tile per CTA.
+//
+// MMA issue order per query tile j (one thread, in-order tensor pipe):
+//     dV(j)   after P^T(j) is in tensor memory       (softmax phase 1)
+//     dK(j)   after dS^T(j) is in shared memory      (softmax phase 2)
+//     S^T(j+1)                                       -> softmax phase 1 of j+1
+//     dQ(j)   into the dP^T columns
+//     dP^T(j+1) after dQ(j) has been read out        -> softmax phase 2 of j+1
+// so the exponentials of tile j+1 overlap dQ(j), its readout and dP^T(j+1).
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
     using L = BwdLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     // The layout needs 1024-byte alignment for the 128-byte swizzle atoms; the
@@ -210,7 +220,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::kQEmpty + s), 1);
         }
         mbar_init(bar(L::kSFull), 1);
-        mbar_init(bar(L::kPFull), 128);
+        mbar_init(bar(L::kPTFull), 128);
+        mbar_init(bar(L::kDPFull), 1);
+        mbar_init(bar(L::kDSFull), 128);
         mbar_init(bar(L::kDQFull), 1);
         mbar_init(bar(L::kDQEmpty), 128);
         mbar_init(bar(L::kAccFull), 1);
@@ -224,6 +236,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_dk);
         prefetch_tmap(&tm_dv);
+        prefetch_tmap(&tm_dqacc);
     }
     tc_fence_before();
     __syncthreads();
@@ -295,51 +308,77 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             constexpr uint32_t idesc_dv = idesc_f16_f32acc(BF16, kBK, D, false, true);     // dV, dK
             constexpr uint32_t idesc_dq = idesc_f16_f32acc(BF16, kBQ, D, true, true);      // dQ
             const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sDS = sbase + L::kDS;
-            bool ok = mbar_wait(bar(L::kKVFull), 0, wctx);
-            for (int jj = 0; jj < nq && ok; ++jj) {
-                const int s = jj & 1;
-                const uint32_t ph = (jj >> 1) & 1;
+            auto issue_st = [&](int s) {   // S^T = K Q^T (both K-major)
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
-                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
-                if (!mbar_wait(bar(L::kQFull + s), ph, wctx)) { ok = false; break; }
-                if (jj > 0 && !mbar_wait(bar(L::kDQEmpty), (jj - 1) & 1, wctx)) { ok = false; break; }
-                tc_fence_after();
-                // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(tmem + L::kColS, smem_desc_sw128(sK + off, 16, 1024),
                                 smem_desc_sw128(sQ + off, 16, 1024), idesc_st, kk > 0);
                 }
+            };
+            auto issue_dpt = [&](int s) {  // dP^T = V dO^T (both K-major)
+                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(tmem + L::kColDP, smem_desc_sw128(sV + off, 16, 1024),
                                 smem_desc_sw128(sDO + off, 16, 1024), idesc_st, kk > 0);
                 }
-                umma_commit(bar(L::kSFull));
-                if (!mbar_wait(bar(L::kPFull), jj & 1, wctx)) { ok = false; break; }
-                tc_fence_after();
+            };
+            bool ok = mbar_wait(bar(L::kKVFull), 0, wctx);
+            if (ok && nq > 0) {
+                ok = mbar_wait(bar(L::kQFull + 0), 0, wctx);
+                if (ok) {
+                    tc_fence_after();
+                    issue_st(0);
+                    umma_commit(bar(L::kSFull));
+                    issue_dpt(0);
+                    umma_commit(bar(L::kDPFull));
+                }
+            }
+            for (int jj = 0; jj < nq && ok; ++jj) {
+                const int s = jj & 1;
+                const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
+                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
+                const bool more = jj + 1 < nq;
                 // dV += P^T dO   (A: P^T in tensor memory; B: dO rows, MN-major)
+                if (!mbar_wait(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
                     umma_f16_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8,
                                 smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_dv,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
                 // dK += dS^T Q   (A: dS^T K-major in shared memory; B: Q rows, MN-major)
+                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
                     umma_f16_ss(tmem + L::kColDK,
                                 smem_desc_sw128(sDS + (kk >> 2) * L::kChunkBytes + (kk & 3) * 32, 16, 1024),
                                 smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_dv,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
-                // dQ_j = dS K   (A: the same dS^T buffer read MN-major; B: K rows, MN-major)
+                if (more) {
+                    const int s2 = (jj + 1) & 1;
+                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_st(s2);
+                    umma_commit(bar(L::kSFull));
+                }
+                // dQ_j = dS K into the dP^T columns (A: dS^T read MN-major; B: K rows, MN-major)
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
                     umma_f16_ss(tmem + L::kColDQ, smem_desc_sw128(sDS + kk * 2048, L::kChunkBytes, 1024),
                                 smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024), idesc_dq, kk > 0);
                 umma_commit(bar(L::kDQFull));
                 if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
+                if (more) {
+                    if (!mbar_wait(bar(L::kDQEmpty), jj & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_dpt((jj + 1) & 1);
+                    umma_commit(bar(L::kDPFull));
+                }
             }
             umma_commit(bar(L::kAccFull));
             umma_commit(bar(L::kDrain));
@@ -349,36 +388,50 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait(bar(L::kDrain), 0, drain);
         }
     } else if (warp >= kReadoutWarp0) {
-        // ===================== dQ readout =====================
+        // ===================== dQ readout: TMEM -> smem -> TMA add =====================
+        // Each warp stages its 32 rows x 64 columns (fp32, two 32x32 boxes with
+        // the 128-byte swizzle) in its quarter of the dS^T buffer, which no MMA
+        // reads between dQ(j) completing and dP^T(j+1) being issued.
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        bool ok = true;
+        uint8_t *stage = smem + L::kDS + wq * 8192;
+        const uint32_t stage_a = sbase + L::kDS + wq * 8192;
         for (int jj = 0; jj < nq; ++jj) {
             const bool got = mbar_wait(bar(L::kDQFull), jj & 1, wctx);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const int q = (j_begin + jj) * kBQ + row;
-            float *dst = p.dq_acc + (static_cast<size_t>(bh) * p.Nq + q) * D;
+            const int q_row0 = (j_begin + jj) * kBQ + wq * 32;
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32dp_x32_wait(tl + L::kColDQ + cc * 32, v);
-                if (q < p.Nq) {
+            for (int half = 0; half < D / 64; ++half) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float4 a = make_float4(__uint_as_float(v[4 * e]) * p.scale,
-                                                     __uint_as_float(v[4 * e + 1]) * p.scale,
-                                                     __uint_as_float(v[4 * e + 2]) * p.scale,
-                                                     __uint_as_float(v[4 * e + 3]) * p.scale);
-                        atomicAdd(reinterpret_cast<float4 *>(dst + cc * 32 + 4 * e), a);
+                for (int box = 0; box < 2; ++box) {
+                    uint32_t v[32];
+                    tmem_ld32dp_x32_wait(tl + L::kColDQ + half * 64 + box * 32, v);
+                    uint8_t *rowp = stage + box * 4096 + lane * 128;
+#pragma unroll
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        const int pos = k4 ^ (lane & 7);
+                        *reinterpret_cast<float4 *>(rowp + pos * 16) =
+                            make_float4(__uint_as_float(v[4 * k4]) * p.scale, __uint_as_float(v[4 * k4 + 1]) * p.scale,
+                                        __uint_as_float(v[4 * k4 + 2]) * p.scale, __uint_as_float(v[4 * k4 + 3]) * p.scale);
                     }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && q_row0 < p.Nq) {
+                    tma_reduce_add_3d(&tm_dqacc, stage_a, half * 64, q_row0, bh);
+                    tma_reduce_add_3d(&tm_dqacc, stage_a + 4096, half * 64 + 32, q_row0, bh);
+                    tma_store_commit();
+                    tma_store_wait_read_all();
+                }
+                __syncwarp();
             }
             tc_fence_before();
             mbar_arrive(bar(L::kDQEmpty));
         }
-        (void)ok;
+        if (lane == 0) tma_store_wait_all();
+        (void)row;
     } else {
         // ===================== recompute P^T, dS^T (one thread per key) =====================
         const int wq = warp & 3;
@@ -394,43 +447,65 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int jj = 0; jj < nq; ++jj) {
             const int s = jj & 1;
             const int q0 = (j_begin + jj) * kBQ;
-            const bool got = mbar_wait(bar(L::kSFull), jj & 1, wctx);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            tc_fence_after();
             const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256;
-            // first query column of this tile this key is masked for: key > q + off
-            const bool diag = CAUSAL && (key > q0 + p.causal_off);
+            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2), to tensor memory
+            {
+                const bool got = mbar_wait(bar(L::kSFull), jj & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            tc_fence_after();
+            const bool diag = CAUSAL && (key > q0 + p.causal_off);   // some column masked
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dpv[32];
+                uint32_t sv[32];
                 tmem_ld32dp_x32_wait(tl + L::kColS + c * 32, sv);
-                tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
                 const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf + c * 32);
-                const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128 + c * 32);
-                float pr[32], dsr[32];
+                uint32_t pp[16];
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 lv = l4[e4];
-                    const float4 dv = d4[e4];
                     const float la[4] = {lv.x, lv.y, lv.z, lv.w};
-                    const float da[4] = {dv.x, dv.y, dv.z, dv.w};
+                    float pe[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int e = 4 * e4 + u;
                         float x = fmaf(__uint_as_float(sv[e]), qk, b2 - la[u]);
                         if (diag && key > q0 + c * 32 + e + p.causal_off) x = neg_inf();
-                        const float pe = ex2_approx(x);
-                        pr[e] = pe;
-                        dsr[e] = pe * (__uint_as_float(dpv[e]) - da[u]);
+                        pe[u] = ex2_approx(x);
                     }
-                }
-                uint32_t pp[16], dd[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    pp[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
-                    dd[e] = pack2<BF16>(dsr[2 * e], dsr[2 * e + 1]);
+                    pp[2 * e4] = pack2<BF16>(pe[0], pe[1]);
+                    pp[2 * e4 + 1] = pack2<BF16>(pe[2], pe[3]);
                 }
                 tmem_st32dp_x16(tl + L::kColS + c * 16, pp);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::kPTFull));
+            // ---- phase 2: dS^T = P^T (dP^T - D), to shared memory
+            {
+                const bool got = mbar_wait(bar(L::kDPFull), jj & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pv[16], dpv[32];
+                tmem_ld32dp_x16_wait(tl + L::kColS + c * 16, pv);
+                tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
+                const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128 + c * 32);
+                uint32_t dd[16];
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 dv = d4[e4];
+                    const float2 p01 = unpack2<BF16>(pv[2 * e4]);
+                    const float2 p23 = unpack2<BF16>(pv[2 * e4 + 1]);
+                    const float ds0 = p01.x * (__uint_as_float(dpv[4 * e4 + 0]) - dv.x);
+                    const float ds1 = p01.y * (__uint_as_float(dpv[4 * e4 + 1]) - dv.y);
+                    const float ds2 = p23.x * (__uint_as_float(dpv[4 * e4 + 2]) - dv.z);
+                    const float ds3 = p23.y * (__uint_as_float(dpv[4 * e4 + 3]) - dv.w);
+                    dd[2 * e4] = pack2<BF16>(ds0, ds1);
+                    dd[2 * e4 + 1] = pack2<BF16>(ds2, ds3);
+                }
                 // dS^T row into shared memory, 128-byte swizzled, 64 queries per chunk
                 const int chunk = (c * 32) / 64;
                 const int k16_base = ((c * 32) % 64) / 8;
@@ -441,10 +516,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
                 }
             }
-            tmem_wait_st();
             tc_fence_before();
             fence_proxy_async_smem();
-            mbar_arrive(bar(L::kPFull));
+            mbar_arrive(bar(L::kDSFull));
         }
 
         // ---- epilogue: dV and scale * dK, 16-bit, via the (now idle) K and V buffers
@@ -513,7 +587,7 @@ cudaError_t launch_dkdv_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
-    kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, p);
+    kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, tm.dqacc, p);
     note_launch();
     return cudaGetLastError();
 }

@@ -42,7 +42,7 @@ struct BwdParams {
 };
 
 struct BwdTensorMaps {
-    CUtensorMap q, k, v, dO, dk, dv;
+    CUtensorMap q, k, v, dO, dk, dv, dqacc;
 };
 
 cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,

@@ -113,6 +113,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, uint32_t src,
                  : "memory");
 }
 
+// Element-wise add of a shared-memory box into global memory (fp32 map),
+// rows outside the tensor are skipped; tracked by the bulk-group counters.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *m, uint32_t src, int x, int y,
+                                                  int z) {
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_store_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

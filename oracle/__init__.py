@@ -63,7 +63,7 @@ def _bind(lib):
     lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                               ip, ctypes.c_int, dp, dp, dp]
+                               ip, ctypes.c_int, ip, ctypes.c_int, dp, dp, dp]
     lib.oracle_bwd.restype = None
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_max_threads.restype = ctypes.c_int
@@ -160,11 +160,14 @@ class Oracle:
         return o, lse
 
 
-    def bwd(self, q, k, v, dO, key_bias=None, causal=False, scale=None, bh_list=None):
+    def bwd(self, q, k, v, dO, key_bias=None, causal=False, scale=None, bh_list=None,
+            rows=None):
         """Exact gradients of L = sum(O * dO) w.r.t. q, k, v in float64.
 
         ``bh_list``: flat (b*H + h) indices to evaluate (None = all).  Returns
         ``(dq, dk, dv)`` of shapes [n, Nq, D], [n, Nk, D], [n, Nk, D].
+        ``rows``: optional query-row subset; only those rows contribute (a
+        bounded sample of the work for timing; None = the full gradient).
         """
         q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
         B, H, Nq, D = q.shape
@@ -177,6 +180,10 @@ class Oracle:
             bh_list = np.arange(B * H)
         bh = np.ascontiguousarray(np.asarray(bh_list, dtype=np.int32))
         n = bh.size
+        rows_arr = None
+        if rows is not None:
+            rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+            assert rows_arr.size == 0 or (rows_arr.min() >= 0 and rows_arr.max() < Nq)
         dq = np.zeros((n, Nq, D))
         dk = np.zeros((n, Nk, D))
         dv = np.zeros((n, Nk, D))
@@ -184,7 +191,9 @@ class Oracle:
             return dq, dk, dv
         self._lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(dO), B, H, Nq,
                            Nk, D, int(bool(causal)), float(scale),
-                           _ptr(bh, ctypes.c_int), n, _ptr(dq), _ptr(dk), _ptr(dv))
+                           _ptr(bh, ctypes.c_int), n, _ptr(rows_arr, ctypes.c_int),
+                           0 if rows_arr is None else rows_arr.size,
+                           _ptr(dq), _ptr(dk), _ptr(dv))
         return dq, dk, dv
 
 

@@ -134,11 +134,15 @@ void oracle_fwd(const double *q, const double *k, const double *v,
  * Outputs dq [n_bh, Nq, D], dk and dv [n_bh, Nk, D] in float64.
  * Row by row: materialise P_i and dP_i, form dS_i, accumulate the three
  * gradients.  No stored O or LSE is used: both are recomputed from scratch.
+ * q_rows == NULL processes every query row; otherwise only the n_q_rows listed
+ * rows contribute (their dQ rows are exact, dK and dV hold only their share):
+ * a bounded sample of the same work, used for CPU timing.
  */
 void oracle_bwd(const double *q, const double *k, const double *v,
                 const double *key_bias, const double *dO, int B, int H, int Nq,
                 int Nk, int D, int causal, double scale, const int *bh_list,
-                int n_bh, double *dq, double *dk, double *dv)
+                int n_bh, const int *q_rows, int n_q_rows, double *dq, double *dk,
+                double *dv)
 {
     (void)B;
 #pragma omp parallel
@@ -160,7 +164,9 @@ void oracle_bwd(const double *q, const double *k, const double *v,
             memset(dqh, 0, sizeof(double) * Nq * D);
             memset(dkh, 0, sizeof(double) * Nk * D);
             memset(dvh, 0, sizeof(double) * Nk * D);
-            for (long i = 0; i < Nq; ++i) {
+            long n_rows = q_rows ? n_q_rows : Nq;
+            for (long r = 0; r < n_rows; ++r) {
+                long i = q_rows ? q_rows[r] : r;
                 /* P_i: the softmax row, rebuilt from scratch */
                 double lse = softmax_row(qh + i * D, kh, bias_b, i, Nq, Nk, D,
                                          causal, scale, p);

@@ -351,6 +351,19 @@ def test_bwd_subset_of_heads(orc):
         assert np.array_equal(a[[4, 1]], b)
 
 
+def test_bwd_row_sample_is_a_partition(orc):
+    """Row-sampled backward: the dQ rows are exact and the dK, dV shares of
+    disjoint row sets add up to the full gradient."""
+    q, k, v, bias = rand_case(1, 2, 9, 11, 4, True, True)
+    do = RNG.standard_normal(q.shape)
+    full = orc.bwd(q, k, v, do, bias, True, 0.5)
+    a = orc.bwd(q, k, v, do, bias, True, 0.5, rows=[0, 3, 4, 8])
+    b = orc.bwd(q, k, v, do, bias, True, 0.5, rows=[1, 2, 5, 6, 7])
+    assert np.allclose(a[0][:, [0, 3, 4, 8]], full[0][:, [0, 3, 4, 8]], rtol=0, atol=1e-14)
+    for t in (1, 2):
+        assert np.allclose(a[t] + b[t], full[t], rtol=1e-13, atol=1e-14)
+
+
 def test_merge_monoid():
     """(+) is associative and commutative with identity (-inf, 0, 0)."""
     rows, D = 6, 4
