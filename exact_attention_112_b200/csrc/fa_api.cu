@@ -85,23 +85,6 @@ int make_map(CUtensorMap *m, const void *ptr, bool bf16, int D, int N, long long
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// 3-D fp32 map over the [B*H, Nq, D] dQ accumulator: 32 x 32 boxes with the
-// 128-byte swizzle, used by the TMA reduce-add of dQ contributions.
-int make_map_f32(CUtensorMap *m, void *ptr, int D, int N, long long BH) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc;
-    int st = get_encoder(&enc);
-    if (st != FA_OK) return st;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
-                          static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(N) * D * 4};
-    cuuint32_t box[3] = {32, 32, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
-}
-
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shared shape/scalar validation of forward and backward.
@@ -188,7 +171,7 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
     if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128)) return 0;
     const size_t rows = static_cast<size_t>(B) * H * Nq;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    return up(rows * sizeof(float)) + up(rows * D * sizeof(float)) + 256;
+    return up(rows * sizeof(float)) + 256;
 }
 
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -219,8 +202,11 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
             return FA_ERR_CUDA;
         return FA_OK;
     }
-    const size_t rows = static_cast<size_t>(BH) * Nq;
-    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    if (Nk == 0) {
+        // no key: every output row is empty, so dQ is zero
+        if (cudaMemsetAsync(dq, 0, static_cast<size_t>(BH) * Nq * D * 2, s) != cudaSuccess) return FA_ERR_CUDA;
+        return FA_OK;
+    }
     fa::BwdParams p;
     p.B = B;
     p.H = H;
@@ -234,20 +220,17 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
     p.o = o;
     p.dO = dO;
     p.Di = static_cast<float *>(workspace);
-    p.dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + up(rows * sizeof(float)));
-    p.dq = dq;
     p.err = err;
     p.timeout_ns = kDefaultTimeoutNs;
     fa::BwdTensorMaps tm;
-    std::memset(&tm, 0, sizeof(tm));
-    if (Nk > 0) {
+    {
         if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
         if ((st = make_map(&tm.dO, dO, bf16, D, Nq, BH, 128)) != FA_OK) return st;
         if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
         if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
         if ((st = make_map(&tm.dk, dk, bf16, D, Nk, BH, 32)) != FA_OK) return st;
         if ((st = make_map(&tm.dv, dv, bf16, D, Nk, BH, 32)) != FA_OK) return st;
-        if ((st = make_map_f32(&tm.dqacc, p.dq_acc, D, Nq, BH)) != FA_OK) return st;
+        if ((st = make_map(&tm.dq, dq, bf16, D, Nq, BH, 32)) != FA_OK) return st;
     }
     cudaError_t e = fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

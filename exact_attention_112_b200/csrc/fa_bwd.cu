@@ -12,27 +12,33 @@
 //   dS = P * (dP - D)  with D_i = sum_j P_ij dP_ij = rowsum(dO * O)
 //   dQ = scale dS K    dK = scale dS^T Q
 //
-// Three kernels on one stream:
-//   1. fa_bwd_pre_kernel     D_i = rowsum(dO * O) (fp32) and dQacc = 0.
-//   2. fa_bwd_dkdv_kernel    one CTA per (b, h, 128-key tile).  For every
-//      query tile j that can see these keys:
-//        S^T  = K Q_j^T, dP^T = V dO_j^T          tcgen05.mma -> tensor memory
-//        P^T  = 2^(S^T qk_scale + bias - LSE_2)    one thread per key row
+// Three kernels on one stream, none of which stores S, P or dS:
+//   1. fa_bwd_pre_kernel   D_i = rowsum(dO * O) (fp32, the caller's workspace).
+//   2. fa_bwd_dkdv_kernel  one CTA per (b, h, 128-key tile); for every query
+//      tile j that can see these keys:
+//        S^T  = K Q_j^T, dP^T = V dO_j^T           tcgen05.mma -> tensor memory
+//        P^T  = 2^(S^T qk_scale + bias - LSE_2)     one thread per key row
 //        dS^T = P^T * (dP^T - D_j)
-//        dV  += P^T dO_j   (P^T from tensor memory)
-//        dK  += dS^T Q_j   (dS^T from shared memory, K-major)
-//        dQ_j = dS K       (the same dS^T buffer read as an MN-major operand)
-//      and a readout warpgroup adds scale * dQ_j into dQacc with TMA bulk
-//      reduce-add (fp32).  dK (x scale) and dV are written once at the end.
-//   3. fa_bwd_dq_convert_kernel  dQ = dQacc cast to the 16-bit type.
+//        dV  += P^T dO_j,  dK += dS^T Q_j           A operands from tensor memory
+//      dK (x scale) and dV are written once at the end.
+//   3. fa_bwd_dq_kernel    one CTA per (b, h, 128-query tile); for every key
+//      tile j it can see: S = Q K_j^T, dP = dO V_j^T, P and dS as above (one
+//      thread per query row), dQ += dS K_j; dQ (x scale) written once.
+// dQ is therefore computed without atomics and is bitwise deterministic; the
+// price is recomputing S and dP in kernel 3 (7 tile products per pair of
+// tiles instead of 5).
 //
-// Tensor memory of the dK/dV kernel (lane = key row, except dQ: lane = query):
-//   cols [0,128)      S^T (fp32); P^T (16-bit pairs) overwrites cols [0,64)
-//   cols [128,256)    dP^T (fp32); dQ_j (fp32) in cols [128,128+D) once dS^T
-//                     has been formed from it
+// Tensor memory of the dK/dV kernel (lane = key row):
+//   cols [0,128)      S^T (fp32); then P^T (16-bit pairs) in [0,64) and
+//                     dS^T (16-bit pairs) in [64,128)
+//   cols [128,256)    dP^T (fp32)
 //   cols [256,256+D)  dV accumulator,  cols [256+D,256+2D) dK accumulator
-// Warp roles (10 warps): 0-3 recompute/gradient, 4-7 dQ readout, 8 TMA
-// producer (also stages LSE and D of each query tile), 9 MMA issuer.
+// Tensor memory of the dQ kernel (lane = query row):
+//   cols [0,128), [128,256)  S of two consecutive key tiles (fp32); dS
+//                            (16-bit pairs) overwrites the first 64 columns
+//   cols [256,384)    dP (fp32),   cols [384,384+D) dQ accumulator
+// Warp roles (6 warps): 0-3 recompute/gradient (one thread per tile row),
+// 4 TMA producer, 5 MMA issuer.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -47,24 +53,22 @@
 namespace fa {
 namespace {
 
-constexpr int kBK = 128;          // keys per CTA tile (MMA M for S^T, dP^T, dV, dK)
-constexpr int kBQ = 128;          // queries per step
-constexpr int kThreads = 320;
-constexpr int kReadoutWarp0 = 4;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kBK = 128;          // keys per tile
+constexpr int kBQ = 128;          // queries per tile
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
-struct BwdLayout {
+struct DkdvLayout {
     static constexpr int kTileBytes = 128 * D * 2;
     static constexpr int kChunkBytes = 128 * 128;     // 128 rows x 64 16-bit values
     static constexpr int kK = 0;
     static constexpr int kV = kK + kTileBytes;
     static constexpr int kQ = kV + kTileBytes;        // 2 stages
     static constexpr int kDO = kQ + 2 * kTileBytes;   // 2 stages
-    static constexpr int kDS = kDO + 2 * kTileBytes;  // dS^T: 128 keys x 128 queries, 16-bit
-    static constexpr int kRow = kDS + 128 * 128 * 2;  // 2 stages x {LSE_2[128], D[128]} f32
+    static constexpr int kRow = kDO + 2 * kTileBytes; // 2 stages x {LSE_2[128], D[128]} f32
     static constexpr int kBar = kRow + 2 * 2 * 128 * 4;
     static constexpr int kKVFull = 0;
     static constexpr int kQFull = 1;    // +stage
@@ -73,15 +77,43 @@ struct BwdLayout {
     static constexpr int kPTFull = 6;
     static constexpr int kDPFull = 7;
     static constexpr int kDSFull = 8;
-    static constexpr int kDQFull = 9;
-    static constexpr int kDQEmpty = 10;
-    static constexpr int kAccFull = 11;
-    static constexpr int kDrain = 12;
-    static constexpr int kNumBars = 13;
+    static constexpr int kAccFull = 9;
+    static constexpr int kDrain = 10;
+    static constexpr int kNumBars = 11;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
+    static constexpr uint32_t kColS = 0, kColP = 0, kColDS = 64, kColDP = 128, kColDV = 256,
+                              kColDK = 256 + D;
+};
+
+template <int D>
+struct DqLayout {
+    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kChunkBytes = 128 * 128;
+    static constexpr int kKStages = 3;
+    static constexpr int kVStages = 2;
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTileBytes;
+    static constexpr int kK = kDO + kTileBytes;                 // kKStages
+    static constexpr int kV = kK + kKStages * kTileBytes;        // kVStages
+    static constexpr int kBias = kV + kVStages * kTileBytes;     // kKStages x 128 f32
+    static constexpr int kBar = kBias + kKStages * 128 * 4;
+    static constexpr int kQFull = 0;
+    static constexpr int kKFull = 1;     // +stage (3)
+    static constexpr int kKEmpty = 4;    // +stage (3)
+    static constexpr int kVFull = 7;     // +stage (2)
+    static constexpr int kVEmpty = 9;    // +stage (2)
+    static constexpr int kSFull = 11;    // +buffer (2)
+    static constexpr int kDPFull = 13;
+    static constexpr int kDSFull = 14;
+    static constexpr int kOFull = 15;
+    static constexpr int kDrain = 16;
+    static constexpr int kNumBars = 17;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColDP = 256, kColDQ = 384;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -110,13 +142,12 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
 }
 
 // ---------------------------------------------------------------------------
-// 1. D_i = rowsum(dO * O) and dQacc = 0.  One warp per row.
+// 1. D_i = rowsum(dO * O).  One warp per row.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
                                                          const uint16_t *__restrict__ dO,
                                                          float *__restrict__ Di,
-                                                         float *__restrict__ dq_acc,
                                                          long long rows) {
     const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -141,46 +172,46 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restr
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) Di[r] = acc;
-        float4 *z = reinterpret_cast<float4 *>(dq_acc + r * D);
-        for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
 // ---------------------------------------------------------------------------
-// 3. dQ = dQacc (already scaled) cast to 16 bits.
+// Shared pieces of the two recompute kernels.
 // ---------------------------------------------------------------------------
-template <bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float4 *__restrict__ acc,
-                                                                uint2 *__restrict__ dq,
-                                                                long long n4) {
-    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-        const float4 a = acc[i];
-        dq[i] = make_uint2(pack2<BF16>(a.x, a.y), pack2<BF16>(a.z, a.w));
+// Write 32 consecutive 16-bit values of one row (16 packed pairs starting at
+// column col0) into a 128-byte-swizzled staging tile of 128-byte rows, 64
+// values per chunk: 16-byte piece k of row r lands at piece k ^ (r % 8).
+__device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0, const uint32_t (&pk)[16],
+                                                int chunk_bytes) {
+    const int chunk = col0 / 64;
+    const int k16_base = (col0 % 64) / 8;
+    uint8_t *rowp = tile + chunk * chunk_bytes + row * 128;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        const int k16 = (k16_base + q4) ^ (row & 7);
+        *reinterpret_cast<uint4 *>(rowp + k16 * 16) =
+            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
     }
 }
 
 // ---------------------------------------------------------------------------
-// 2. dK, dV (and dQ contributions) for one 128-key tile per CTA.
+// 2. dK, dV for one 128-key tile per CTA.
 //
 // MMA issue order per query tile j (one thread, in-order tensor pipe):
-//     dV(j)   after P^T(j) is in tensor memory       (softmax phase 1)
-//     dK(j)   after dS^T(j) is in shared memory      (softmax phase 2)
-//     S^T(j+1)                                       -> softmax phase 1 of j+1
-//     dQ(j)   into the dP^T columns
-//     dP^T(j+1) after dQ(j) has been read out        -> softmax phase 2 of j+1
-// so the exponentials of tile j+1 overlap dQ(j), its readout and dP^T(j+1).
+//     dV(j)      once P^T(j) is in tensor memory   (recompute phase 1)
+//     dK(j)      once dS^T(j) is in tensor memory  (recompute phase 2)
+//     S^T(j+1), dP^T(j+1)
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                   const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
-    using L = BwdLayout<D>;
+                   const BwdParams p) {
+    using L = DkdvLayout<D>;
     extern __shared__ uint8_t smem_raw[];
-    // The layout needs 1024-byte alignment for the 128-byte swizzle atoms; the
-    // dynamic shared window starts aligned when no static shared memory is used.
+    // 1024-byte alignment is needed by the 128-byte swizzle atoms; the dynamic
+    // shared window starts aligned when the kernel has no static shared memory.
     if ((smem_u32(smem_raw) & 1023u) != 0) {
         if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
         return;
@@ -190,7 +221,6 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -223,8 +253,6 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar(L::kPTFull), 128);
         mbar_init(bar(L::kDPFull), 1);
         mbar_init(bar(L::kDSFull), 128);
-        mbar_init(bar(L::kDQFull), 1);
-        mbar_init(bar(L::kDQEmpty), 128);
         mbar_init(bar(L::kAccFull), 1);
         mbar_init(bar(L::kDrain), 1);
         fence_mbar_init();
@@ -236,18 +264,17 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_dk);
         prefetch_tmap(&tm_dv);
-        prefetch_tmap(&tm_dqacc);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
-    const float *lse_bh = p.lse + static_cast<size_t>(bh) * p.Nq;
-    const float *di_bh = p.Di + static_cast<size_t>(bh) * p.Nq;
 
     if (warp == kProducerWarp) {
         // ===================== producer =====================
+        const float *lse_bh = p.lse + static_cast<size_t>(bh) * p.Nq;
+        const float *di_bh = p.Di + static_cast<size_t>(bh) * p.Nq;
         bool ok = true;
         int issued = 0;
         if (lane == 0) {
@@ -305,79 +332,60 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // ===================== MMA issuer =====================
         if (lane == 0) {
             constexpr uint32_t idesc_st = idesc_f16_f32acc(BF16, kBK, kBQ, false, false);  // S^T, dP^T
-            constexpr uint32_t idesc_dv = idesc_f16_f32acc(BF16, kBK, D, false, true);     // dV, dK
-            constexpr uint32_t idesc_dq = idesc_f16_f32acc(BF16, kBQ, D, true, true);      // dQ
-            const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sDS = sbase + L::kDS;
-            auto issue_st = [&](int s) {   // S^T = K Q^T (both K-major)
+            constexpr uint32_t idesc_acc = idesc_f16_f32acc(BF16, kBK, D, false, true);    // dV, dK
+            const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
+            auto issue_st_dpt = [&](int s) {   // S^T = K Q^T, dP^T = V dO^T (all K-major)
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
+                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(tmem + L::kColS, smem_desc_sw128(sK + off, 16, 1024),
                                 smem_desc_sw128(sQ + off, 16, 1024), idesc_st, kk > 0);
                 }
-            };
-            auto issue_dpt = [&](int s) {  // dP^T = V dO^T (both K-major)
-                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
+                umma_commit(bar(L::kSFull));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(tmem + L::kColDP, smem_desc_sw128(sV + off, 16, 1024),
                                 smem_desc_sw128(sDO + off, 16, 1024), idesc_st, kk > 0);
                 }
+                umma_commit(bar(L::kDPFull));
             };
             bool ok = mbar_wait(bar(L::kKVFull), 0, wctx);
             if (ok && nq > 0) {
                 ok = mbar_wait(bar(L::kQFull + 0), 0, wctx);
                 if (ok) {
                     tc_fence_after();
-                    issue_st(0);
-                    umma_commit(bar(L::kSFull));
-                    issue_dpt(0);
-                    umma_commit(bar(L::kDPFull));
+                    issue_st_dpt(0);
                 }
             }
             for (int jj = 0; jj < nq && ok; ++jj) {
                 const int s = jj & 1;
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
                 const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
-                const bool more = jj + 1 < nq;
                 // dV += P^T dO   (A: P^T in tensor memory; B: dO rows, MN-major)
                 if (!mbar_wait(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8,
-                                smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_dv,
+                    umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + kk * 8,
+                                smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
-                // dK += dS^T Q   (A: dS^T K-major in shared memory; B: Q rows, MN-major)
+                // dK += dS^T Q   (A: dS^T in tensor memory; B: Q rows, MN-major)
                 if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ss(tmem + L::kColDK,
-                                smem_desc_sw128(sDS + (kk >> 2) * L::kChunkBytes + (kk & 3) * 32, 16, 1024),
-                                smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_dv,
+                    umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + kk * 8,
+                                smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
-                if (more) {
+                if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
+                if (jj + 1 < nq) {
                     const int s2 = (jj + 1) & 1;
                     if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
                     tc_fence_after();
-                    issue_st(s2);
-                    umma_commit(bar(L::kSFull));
-                }
-                // dQ_j = dS K into the dP^T columns (A: dS^T read MN-major; B: K rows, MN-major)
-#pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    umma_f16_ss(tmem + L::kColDQ, smem_desc_sw128(sDS + kk * 2048, L::kChunkBytes, 1024),
-                                smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024), idesc_dq, kk > 0);
-                umma_commit(bar(L::kDQFull));
-                if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
-                if (more) {
-                    if (!mbar_wait(bar(L::kDQEmpty), jj & 1, wctx)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_dpt((jj + 1) & 1);
-                    umma_commit(bar(L::kDPFull));
+                    issue_st_dpt(s2);
                 }
             }
             umma_commit(bar(L::kAccFull));
@@ -387,51 +395,6 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             drain.abort_flag = &zero;
             mbar_wait(bar(L::kDrain), 0, drain);
         }
-    } else if (warp >= kReadoutWarp0) {
-        // ===================== dQ readout: TMEM -> smem -> TMA add =====================
-        // Each warp stages its 32 rows x 64 columns (fp32, two 32x32 boxes with
-        // the 128-byte swizzle) in its quarter of the dS^T buffer, which no MMA
-        // reads between dQ(j) completing and dP^T(j+1) being issued.
-        const int wq = warp & 3;
-        const int row = wq * 32 + lane;
-        const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        uint8_t *stage = smem + L::kDS + wq * 8192;
-        const uint32_t stage_a = sbase + L::kDS + wq * 8192;
-        for (int jj = 0; jj < nq; ++jj) {
-            const bool got = mbar_wait(bar(L::kDQFull), jj & 1, wctx);
-            if (!__all_sync(0xffffffffu, got)) break;
-            tc_fence_after();
-            const int q_row0 = (j_begin + jj) * kBQ + wq * 32;
-#pragma unroll
-            for (int half = 0; half < D / 64; ++half) {
-#pragma unroll
-                for (int box = 0; box < 2; ++box) {
-                    uint32_t v[32];
-                    tmem_ld32dp_x32_wait(tl + L::kColDQ + half * 64 + box * 32, v);
-                    uint8_t *rowp = stage + box * 4096 + lane * 128;
-#pragma unroll
-                    for (int k4 = 0; k4 < 8; ++k4) {
-                        const int pos = k4 ^ (lane & 7);
-                        *reinterpret_cast<float4 *>(rowp + pos * 16) =
-                            make_float4(__uint_as_float(v[4 * k4]) * p.scale, __uint_as_float(v[4 * k4 + 1]) * p.scale,
-                                        __uint_as_float(v[4 * k4 + 2]) * p.scale, __uint_as_float(v[4 * k4 + 3]) * p.scale);
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && q_row0 < p.Nq) {
-                    tma_reduce_add_3d(&tm_dqacc, stage_a, half * 64, q_row0, bh);
-                    tma_reduce_add_3d(&tm_dqacc, stage_a + 4096, half * 64 + 32, q_row0, bh);
-                    tma_store_commit();
-                    tma_store_wait_read_all();
-                }
-                __syncwarp();
-            }
-            tc_fence_before();
-            mbar_arrive(bar(L::kDQEmpty));
-        }
-        if (lane == 0) tma_store_wait_all();
-        (void)row;
     } else {
         // ===================== recompute P^T, dS^T (one thread per key) =====================
         const int wq = warp & 3;
@@ -442,46 +405,45 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         float b2 = key < p.Nk ? 0.f : neg_inf();
         if (HAS_BIAS && key < p.Nk)
             b2 = __ldg(p.bias + static_cast<size_t>(bh / p.H) * p.Nk + key) * kLog2e;
-        uint8_t *ds_row = smem + L::kDS + row * 128;
         bool ok = true;
         for (int jj = 0; jj < nq; ++jj) {
             const int s = jj & 1;
             const int q0 = (j_begin + jj) * kBQ;
             const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256;
-            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2), to tensor memory
+            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2) -> tensor memory (16-bit)
             {
                 const bool got = mbar_wait(bar(L::kSFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
             const bool diag = CAUSAL && (key > q0 + p.causal_off);   // some column masked
+            float pr[128];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t sv[32];
                 tmem_ld32dp_x32_wait(tl + L::kColS + c * 32, sv);
                 const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf + c * 32);
-                uint32_t pp[16];
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 lv = l4[e4];
                     const float la[4] = {lv.x, lv.y, lv.z, lv.w};
-                    float pe[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int e = 4 * e4 + u;
                         float x = fmaf(__uint_as_float(sv[e]), qk, b2 - la[u]);
                         if (diag && key > q0 + c * 32 + e + p.causal_off) x = neg_inf();
-                        pe[u] = ex2_approx(x);
+                        pr[c * 32 + e] = ex2_approx(x);
                     }
-                    pp[2 * e4] = pack2<BF16>(pe[0], pe[1]);
-                    pp[2 * e4 + 1] = pack2<BF16>(pe[2], pe[3]);
                 }
-                tmem_st32dp_x16(tl + L::kColS + c * 16, pp);
+                uint32_t pp[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pp[e] = pack2<BF16>(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
+                tmem_st32dp_x16(tl + L::kColP + c * 16, pp);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::kPTFull));
-            // ---- phase 2: dS^T = P^T (dP^T - D), to shared memory
+            // ---- phase 2: dS^T = P^T (dP^T - D) -> tensor memory (16-bit)
             {
                 const bool got = mbar_wait(bar(L::kDPFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -489,35 +451,23 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t pv[16], dpv[32];
-                tmem_ld32dp_x16_wait(tl + L::kColS + c * 16, pv);
+                uint32_t dpv[32];
                 tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
                 const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128 + c * 32);
                 uint32_t dd[16];
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 dv = d4[e4];
-                    const float2 p01 = unpack2<BF16>(pv[2 * e4]);
-                    const float2 p23 = unpack2<BF16>(pv[2 * e4 + 1]);
-                    const float ds0 = p01.x * (__uint_as_float(dpv[4 * e4 + 0]) - dv.x);
-                    const float ds1 = p01.y * (__uint_as_float(dpv[4 * e4 + 1]) - dv.y);
-                    const float ds2 = p23.x * (__uint_as_float(dpv[4 * e4 + 2]) - dv.z);
-                    const float ds3 = p23.y * (__uint_as_float(dpv[4 * e4 + 3]) - dv.w);
-                    dd[2 * e4] = pack2<BF16>(ds0, ds1);
-                    dd[2 * e4 + 1] = pack2<BF16>(ds2, ds3);
+                    const int e = c * 32 + 4 * e4;
+                    dd[2 * e4] = pack2<BF16>(pr[e] * (__uint_as_float(dpv[4 * e4]) - dv.x),
+                                             pr[e + 1] * (__uint_as_float(dpv[4 * e4 + 1]) - dv.y));
+                    dd[2 * e4 + 1] = pack2<BF16>(pr[e + 2] * (__uint_as_float(dpv[4 * e4 + 2]) - dv.z),
+                                                 pr[e + 3] * (__uint_as_float(dpv[4 * e4 + 3]) - dv.w));
                 }
-                // dS^T row into shared memory, 128-byte swizzled, 64 queries per chunk
-                const int chunk = (c * 32) / 64;
-                const int k16_base = ((c * 32) % 64) / 8;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int k16 = (k16_base + q4) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(ds_row + chunk * L::kChunkBytes + k16 * 16) =
-                        make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
-                }
+                tmem_st32dp_x16(tl + L::kColDS + c * 16, dd);
             }
+            tmem_wait_st();
             tc_fence_before();
-            fence_proxy_async_smem();
             mbar_arrive(bar(L::kDSFull));
         }
 
@@ -546,15 +496,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-                    const int chunk = (cc * 32) / 64;
-                    const int k16_base = ((cc * 32) % 64) / 8;
-                    uint8_t *rowp = stage + chunk * L::kChunkBytes + row * 128;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int k16 = (k16_base + q4) ^ (row & 7);
-                        *reinterpret_cast<uint4 *>(rowp + k16 * 16) =
-                            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-                    }
+                    stage_row_sw128(stage, row, cc * 32, pk, L::kChunkBytes);
                 }
             }
             fence_proxy_async_smem();
@@ -580,50 +522,391 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
+// ---------------------------------------------------------------------------
+// 3. dQ for one 128-query tile per CTA.
+//
+// MMA issue order per key tile j:
+//     dQ(j)      once dS(j) is in tensor memory (S buffer j % 2)
+//     dP(j+1)    (the dP columns were read by the recompute of j)
+//     S(j+2)     into S buffer j % 2
+// so the exponentials of tile j+1 (whose S was computed one step earlier)
+// overlap dQ(j) and dP(j+1).
+// ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-cudaError_t launch_dkdv_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
-    using L = BwdLayout<D>;
-    auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-    if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
-    kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, tm.dqacc, p);
-    note_launch();
-    return cudaGetLastError();
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+    using L = DqLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
+        return;
+    }
+    uint8_t *smem = smem_raw;
+    const uint32_t sbase = smem_u32(smem);
+    auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: query tiles that see the most key tiles come first
+    const int BH = p.B * p.H;
+    const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
+    const int qt = (n_q_all - 1) - blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
+    const int q0 = qt * kBQ;
+    const int n_kv_all = (p.Nk + kBK - 1) / kBK;
+    int n = n_kv_all;
+    if (CAUSAL) {
+        const int last_row = min(q0 + kBQ - 1, p.Nq - 1);
+        const int lim = last_row + p.causal_off;
+        n = lim < 0 ? 0 : min(n_kv_all, lim / kBK + 1);
+    }
+
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(L::kQFull), 1);
+        for (int s = 0; s < L::kKStages; ++s) {
+            mbar_init(bar(L::kKFull + s), HAS_BIAS ? 2 : 1);
+            mbar_init(bar(L::kKEmpty + s), 1);
+        }
+        for (int s = 0; s < L::kVStages; ++s) {
+            mbar_init(bar(L::kVFull + s), 1);
+            mbar_init(bar(L::kVEmpty + s), 1);
+        }
+        mbar_init(bar(L::kSFull + 0), 1);
+        mbar_init(bar(L::kSFull + 1), 1);
+        mbar_init(bar(L::kDPFull), 1);
+        mbar_init(bar(L::kDSFull), 128);
+        mbar_init(bar(L::kOFull), 1);
+        mbar_init(bar(L::kDrain), 1);
+        fence_mbar_init();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_dq);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
+
+    if (warp == kProducerWarp) {
+        // ===================== producer =====================
+        const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(bh / p.H) * p.Nk : nullptr;
+        bool ok = true;
+        int k_issued = 0, v_issued = 0;
+        if (lane == 0 && n > 0) {
+            mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTileBytes);
+            for (int c = 0; c < D / 64; ++c) {
+                tma_load_3d(sbase + L::kQ + c * L::kChunkBytes, &tm_q, bar(L::kQFull), c * 64, q0, bh);
+                tma_load_3d(sbase + L::kDO + c * L::kChunkBytes, &tm_do, bar(L::kQFull), c * 64, q0, bh);
+            }
+        }
+        // K runs up to two tiles ahead of V (K_j is needed by S(j) one step
+        // before V_j is needed by dP(j)).
+        for (int j = 0; j < n && ok; ++j) {
+            const int ks = j % L::kKStages;
+            const uint32_t kph = (j / L::kKStages) & 1;
+            {
+                const bool got = mbar_wait(bar(L::kKEmpty + ks), kph ^ 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(L::kKFull + ks), L::kTileBytes);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(sbase + L::kK + ks * L::kTileBytes + c * L::kChunkBytes, &tm_k,
+                                bar(L::kKFull + ks), c * 64, j * kBK, bh);
+            }
+            if constexpr (HAS_BIAS) {
+                float *bs = reinterpret_cast<float *>(smem + L::kBias) + ks * 128;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = j * kBK + lane * 4 + e;
+                    bs[lane * 4 + e] = key < p.Nk ? __ldg(bias_b + key) * kLog2e : neg_inf();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kKFull + ks));
+            }
+            k_issued = j + 1;
+            if (j >= 1) {
+                const int jv = j - 1;
+                const int vs = jv % L::kVStages;
+                const uint32_t vph = (jv / L::kVStages) & 1;
+                const bool got = mbar_wait(bar(L::kVEmpty + vs), vph ^ 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
+                                    bar(L::kVFull + vs), c * 64, jv * kBK, bh);
+                }
+                v_issued = jv + 1;
+            }
+        }
+        if (ok && n > 0) {   // the last V tile
+            const int jv = n - 1;
+            const int vs = jv % L::kVStages;
+            const uint32_t vph = (jv / L::kVStages) & 1;
+            const bool got = mbar_wait(bar(L::kVEmpty + vs), vph ^ 1, wctx);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
+                                    bar(L::kVFull + vs), c * 64, jv * kBK, bh);
+                }
+                v_issued = n;
+            }
+        }
+        if (!ok && lane == 0) {
+            WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
+            volatile int zero = 0;
+            drain.abort_flag = &zero;
+            if (n > 0) mbar_wait(bar(L::kQFull), 0, drain);
+            for (int j = (k_issued > 3 ? k_issued - 3 : 0); j < k_issued; ++j)
+                mbar_wait(bar(L::kKFull + j % L::kKStages), (j / L::kKStages) & 1, drain);
+            for (int j = (v_issued > 2 ? v_issued - 2 : 0); j < v_issued; ++j)
+                mbar_wait(bar(L::kVFull + j % L::kVStages), (j / L::kVStages) & 1, drain);
+        }
+    } else if (warp == kMmaWarp) {
+        // ===================== MMA issuer =====================
+        if (lane == 0 && n > 0) {
+            constexpr uint32_t idesc_s = idesc_f16_f32acc(BF16, kBQ, kBK, false, false);   // S, dP
+            constexpr uint32_t idesc_dq = idesc_f16_f32acc(BF16, kBQ, D, false, true);     // dQ
+            const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO;
+            auto issue_s = [&](int j) {        // S_j = Q K_j^T into buffer j % 2
+                const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
+                const uint32_t d = tmem + ((j & 1) ? L::kColS1 : L::kColS0);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                    umma_f16_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024),
+                                idesc_s, kk > 0);
+                }
+                umma_commit(bar(L::kSFull + (j & 1)));
+            };
+            auto issue_dp = [&](int j) {       // dP_j = dO V_j^T
+                const uint32_t sV = sbase + L::kV + (j % L::kVStages) * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                    umma_f16_ss(tmem + L::kColDP, smem_desc_sw128(sDO + off, 16, 1024),
+                                smem_desc_sw128(sV + off, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(bar(L::kDPFull));
+            };
+            bool ok = mbar_wait(bar(L::kQFull), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+                ok = mbar_wait(bar(L::kVFull + 0), 0, wctx);
+            }
+            if (ok) {
+                tc_fence_after();
+                issue_dp(0);
+                if (2 < n) umma_commit(bar(L::kVEmpty + 0));
+                if (n > 1) {
+                    ok = mbar_wait(bar(L::kKFull + 1), 0, wctx);
+                    if (ok) {
+                        tc_fence_after();
+                        issue_s(1);
+                    }
+                }
+            }
+            for (int j = 0; j < n && ok; ++j) {
+                // dQ += dS_j K_j  (A: dS in tensor memory; B: K rows, MN-major)
+                if (!mbar_wait(bar(L::kDSFull), j & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
+                const uint32_t a = tmem + ((j & 1) ? L::kColS1 : L::kColS0);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    umma_f16_ts(tmem + L::kColDQ, a + kk * 8, smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024),
+                                idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                if (j + 3 < n) umma_commit(bar(L::kKEmpty + j % L::kKStages));
+                if (j + 1 < n) {
+                    const int jv = j + 1;
+                    if (!mbar_wait(bar(L::kVFull + jv % L::kVStages), (jv / L::kVStages) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_dp(jv);
+                    if (jv + 2 < n) umma_commit(bar(L::kVEmpty + jv % L::kVStages));
+                }
+                if (j + 2 < n) {
+                    const int js = j + 2;
+                    if (!mbar_wait(bar(L::kKFull + js % L::kKStages), (js / L::kKStages) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_s(js);
+                }
+            }
+            umma_commit(bar(L::kOFull));
+            umma_commit(bar(L::kDrain));
+            WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
+            volatile int zero = 0;
+            drain.abort_flag = &zero;
+            mbar_wait(bar(L::kDrain), 0, drain);
+        }
+    } else {
+        // ===================== recompute P, dS (one thread per query row) =====================
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const int q = q0 + row;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const float qk = p.qk_scale_log2;
+        float lse2 = pos_inf(), di = 0.f;
+        if (q < p.Nq) {
+            const float l = __ldg(p.lse + static_cast<size_t>(bh) * p.Nq + q);
+            lse2 = (l == neg_inf()) ? pos_inf() : l * kLog2e;
+            di = __ldg(p.Di + static_cast<size_t>(bh) * p.Nq + q);
+        }
+        // last key this row may see
+        const int lim = CAUSAL ? min(q + p.causal_off, p.Nk - 1) : p.Nk - 1;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int kv0 = j * kBK;
+            const uint32_t tS = tl + ((j & 1) ? L::kColS1 : L::kColS0);
+            {
+                const bool got = mbar_wait(bar(L::kSFull + (j & 1)), (j >> 1) & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            tc_fence_after();
+            // ---- P = 2^(S qk + bias - LSE_2), kept in registers
+            float pr[128];
+            const float *bs = reinterpret_cast<const float *>(smem + L::kBias) + (j % L::kKStages) * 128;
+            const bool edge = kv0 + kBK - 1 > lim;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32];
+                tmem_ld32dp_x32_wait(tS + c * 32, sv);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float x;
+                    if constexpr (HAS_BIAS)
+                        x = fmaf(__uint_as_float(sv[e]), qk, bs[c * 32 + e] - lse2);
+                    else
+                        x = fmaf(__uint_as_float(sv[e]), qk, -lse2);
+                    if (edge && kv0 + c * 32 + e > lim) x = neg_inf();
+                    pr[c * 32 + e] = ex2_approx(x);
+                }
+            }
+            // ---- dS = P (dP - D) -> tensor memory (16-bit), over the S columns
+            {
+                const bool got = mbar_wait(bar(L::kDPFull), j & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t dpv[32];
+                tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
+                uint32_t dd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    dd[e] = pack2<BF16>(pr[c * 32 + 2 * e] * (__uint_as_float(dpv[2 * e]) - di),
+                                        pr[c * 32 + 2 * e + 1] * (__uint_as_float(dpv[2 * e + 1]) - di));
+                tmem_st32dp_x16(tS + c * 16, dd);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::kDSFull));
+        }
+        // ---- epilogue: dQ = scale * acc, 16-bit, staged in the (idle) Q buffer
+        if (ok && n > 0) {
+            const bool got = mbar_wait(bar(L::kOFull), 0, wctx);
+            ok = __all_sync(0xffffffffu, got);
+            tc_fence_after();
+        }
+        if (ok) {
+            uint8_t *stage = smem + L::kQ;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                if (n > 0) {
+                    tmem_ld32dp_x32_wait(tl + L::kColDQ + cc * 32, v);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * p.scale, __uint_as_float(v[2 * e + 1]) * p.scale);
+                stage_row_sw128(stage, row, cc * 32, pk, L::kChunkBytes);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int row0 = q0 + wq * 32;
+            if (lane == 0 && row0 < p.Nq) {
+                for (int c = 0; c < D / 64; ++c)
+                    tma_store_3d(&tm_dq, sbase + L::kQ + c * L::kChunkBytes + wq * 32 * 128, c * 64, row0, bh);
+                tma_store_commit();
+                tma_store_wait_all();
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
+    {
+        using L = DkdvLayout<D>;
+        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
+        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, p);
+        note_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        using L = DqLayout<D>;
+        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
+        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dq, p);
+        note_launch();
+        return cudaGetLastError();
+    }
 }
 
 template <int D, bool BF16>
 cudaError_t launch_bwd_d(const BwdTensorMaps &tm, const BwdParams &p, bool causal, bool bias,
                          cudaStream_t s) {
-    // 1. pre-pass
+    // 1. D_i
     {
         const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
         const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
         fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
-                                                         static_cast<const uint16_t *>(p.dO), p.Di,
-                                                         p.dq_acc, rows);
+                                                         static_cast<const uint16_t *>(p.dO), p.Di, rows);
         note_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    // 2. dK, dV and dQ accumulation
-    if (p.Nk > 0) {
-        cudaError_t e;
-        if (causal)
-            e = bias ? launch_dkdv_t<D, BF16, true, true>(tm, p, s) : launch_dkdv_t<D, BF16, true, false>(tm, p, s);
-        else
-            e = bias ? launch_dkdv_t<D, BF16, false, true>(tm, p, s) : launch_dkdv_t<D, BF16, false, false>(tm, p, s);
-        if (e != cudaSuccess) return e;
-    }
-    // 3. dQ to 16 bits
-    {
-        const long long n4 = static_cast<long long>(p.B) * p.H * p.Nq * D / 4;
-        const unsigned grid = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148LL * 16));
-        fa_bwd_dq_convert_kernel<BF16><<<grid, 256, 0, s>>>(reinterpret_cast<const float4 *>(p.dq_acc),
-                                                             static_cast<uint2 *>(p.dq), n4);
-        note_launch();
-        return cudaGetLastError();
-    }
+    // 2. dK, dV and 3. dQ
+    if (causal)
+        return bias ? launch_grad_t<D, BF16, true, true>(tm, p, s) : launch_grad_t<D, BF16, true, false>(tm, p, s);
+    return bias ? launch_grad_t<D, BF16, false, true>(tm, p, s) : launch_grad_t<D, BF16, false, false>(tm, p, s);
 }
 
 }  // namespace

@@ -35,14 +35,12 @@ struct BwdParams {
     const float *lse;              // [B*H, Nq] from the forward
     const void *o, *dO;            // [B*H, Nq, D] 16-bit
     float *Di;                     // workspace: [B*H*Nq]
-    float *dq_acc;                 // workspace: [B*H*Nq, D] fp32
-    void *dq;                      // [B*H, Nq, D] 16-bit output
     int *err;
     unsigned long long timeout_ns;
 };
 
 struct BwdTensorMaps {
-    CUtensorMap q, k, v, dO, dk, dv, dqacc;
+    CUtensorMap q, k, v, dO, dk, dv, dq;
 };
 
 cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,

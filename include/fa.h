@@ -79,14 +79,15 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 
 /*
  * Bytes of device scratch fa_bwd() needs for these sizes: the per-row term
- * D_i = rowsum(dO * O) (float32) and a float32 dQ accumulator.
+ * D_i = rowsum(dO * O), one float32 per query row (O(n) memory).
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D);
 
 /*
  * Backward pass of L = sum(O * dO): writes dq, dk, dv (dtype, same layouts as
  * q, k, v).  o and lse must be the outputs of fa_fwd() for the same inputs.
- * Scores and probabilities are recomputed tile by tile from q, k and lse.
+ * Scores and probabilities are recomputed tile by tile from q, k and lse;
+ * no atomics are used, so the result is bitwise reproducible.
  * workspace: device memory of at least fa_bwd_workspace_bytes() bytes,
  * 16-byte aligned, owned by the caller; its contents on entry do not matter.
  * The mask and key_bias receive no gradient.

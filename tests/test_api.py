@@ -82,8 +82,8 @@ def test_workspace_size(L):
     B, H, N, D = 2, 32, 4096, 128
     ws = fa.fa_bwd_workspace_bytes(B, H, N, N, D)
     rows = B * H * N
-    assert ws >= rows * 4 + rows * D * 4
-    assert ws < rows * 4 + rows * D * 4 + 4096
+    assert ws >= rows * 4
+    assert ws < rows * 4 + 4096
     assert fa.fa_bwd_workspace_bytes(1, 1, 256, 256, 96) == 0
 
 
