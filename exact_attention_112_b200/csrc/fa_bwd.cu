@@ -29,16 +29,19 @@
 // tiles instead of 5).
 //
 // Tensor memory of the dK/dV kernel (lane = key row):
-//   cols [0,128)      S^T (fp32); then P^T (16-bit pairs) in [0,64) and
-//                     dS^T (16-bit pairs) in [64,128)
-//   cols [128,256)    dP^T (fp32)
+//   cols [0,128)      S^T (fp32)
+//   cols [128,256)    dP^T (fp32); then, in the 64 columns each recompute
+//                     warpgroup read, P^T (16-bit pairs) in the first 32 and
+//                     dS^T (16-bit pairs) in the next 32
 //   cols [256,256+D)  dV accumulator,  cols [256+D,256+2D) dK accumulator
 // Tensor memory of the dQ kernel (lane = query row):
 //   cols [0,128), [128,256)  S of two consecutive key tiles (fp32); dS
-//                            (16-bit pairs) overwrites the first 64 columns
+//                            (16-bit pairs) overwrites the first 32 of each
+//                            warpgroup's 64 columns
 //   cols [256,384)    dP (fp32),   cols [384,384+D) dQ accumulator
-// Warp roles (6 warps): 0-3 recompute/gradient (one thread per tile row),
-// 4 TMA producer, 5 MMA issuer.
+// Warp roles (10 warps): 0-7 recompute/gradient (one thread per tile row and
+// half of the tile's columns: warpgroup g owns columns [64g, 64g+64)), 8 TMA
+// producer, 9 MMA issuer.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -55,9 +58,10 @@ namespace {
 
 constexpr int kBK = 128;          // keys per tile
 constexpr int kBQ = 128;          // queries per tile
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kRecompute = 256;   // two warpgroups, each owning 64 of a tile's 128 columns
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -83,7 +87,11 @@ struct DkdvLayout {
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0, kColP = 0, kColDS = 64, kColDP = 128, kColDV = 256,
+    // Each recompute warpgroup g writes its 16-bit results only into the dP^T
+    // columns it has read itself, 128 + [64g, 64g+64): P^T pairs in the first
+    // 32 of them, dS^T pairs in the next 32.  The S^T columns are therefore
+    // free as soon as phase 1 has loaded them.
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 128, kColDS = 160, kColDV = 256,
                               kColDK = 256 + D;
 };
 
@@ -198,9 +206,11 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 // 2. dK, dV for one 128-key tile per CTA.
 //
 // MMA issue order per query tile j (one thread, in-order tensor pipe):
-//     dV(j)      once P^T(j) is in tensor memory   (recompute phase 1)
-//     dK(j)      once dS^T(j) is in tensor memory  (recompute phase 2)
-//     S^T(j+1), dP^T(j+1)
+//     S^T(j+1)           once phase 1 of j has loaded S^T(j) into registers
+//     dV(j), dK(j)       once phase 2 of j has put P^T, dS^T in tensor memory
+//     dP^T(j+1)
+// so S^T(j+1) is computed while the recompute warps run phase 2 of j, and
+// they go straight on to phase 1 of j+1.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -250,9 +260,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::kQEmpty + s), 1);
         }
         mbar_init(bar(L::kSFull), 1);
-        mbar_init(bar(L::kPTFull), 128);
+        mbar_init(bar(L::kPTFull), kRecompute);
         mbar_init(bar(L::kDPFull), 1);
-        mbar_init(bar(L::kDSFull), 128);
+        mbar_init(bar(L::kDSFull), kRecompute);
         mbar_init(bar(L::kAccFull), 1);
         mbar_init(bar(L::kDrain), 1);
         fence_mbar_init();
@@ -334,9 +344,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             constexpr uint32_t idesc_st = idesc_f16_f32acc(BF16, kBK, kBQ, false, false);  // S^T, dP^T
             constexpr uint32_t idesc_acc = idesc_f16_f32acc(BF16, kBK, D, false, true);    // dV, dK
             const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
-            auto issue_st_dpt = [&](int s) {   // S^T = K Q^T, dP^T = V dO^T (all K-major)
+            auto issue_st = [&](int s) {    // S^T = K Q^T (both K-major)
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
-                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
@@ -344,6 +353,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 smem_desc_sw128(sQ + off, 16, 1024), idesc_st, kk > 0);
                 }
                 umma_commit(bar(L::kSFull));
+            };
+            auto issue_dpt = [&](int s) {   // dP^T = V dO^T (both K-major)
+                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
@@ -357,36 +369,39 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ok = mbar_wait(bar(L::kQFull + 0), 0, wctx);
                 if (ok) {
                     tc_fence_after();
-                    issue_st_dpt(0);
+                    issue_st(0);
+                    issue_dpt(0);
                 }
             }
             for (int jj = 0; jj < nq && ok; ++jj) {
                 const int s = jj & 1;
+                const int s2 = (jj + 1) & 1;
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
                 const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
-                // dV += P^T dO   (A: P^T in tensor memory; B: dO rows, MN-major)
+                // S^T(j+1) into the S^T columns, free once phase 1 of j has read them
                 if (!mbar_wait(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
+                if (jj + 1 < nq) {
+                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_st(s2);
+                }
+                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
+                // dV += P^T dO   (A: P^T in tensor memory; B: dO rows, MN-major)
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + kk * 8,
+                    umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + (kk >> 2) * 64 + (kk & 3) * 8,
                                 smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
                 // dK += dS^T Q   (A: dS^T in tensor memory; B: Q rows, MN-major)
-                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
-                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + kk * 8,
+                    umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + (kk >> 2) * 64 + (kk & 3) * 8,
                                 smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
                 if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
-                if (jj + 1 < nq) {
-                    const int s2 = (jj + 1) & 1;
-                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_st_dpt(s2);
-                }
+                // dP^T(j+1) over the P^T / dS^T of j (read by dV(j), dK(j) just before)
+                if (jj + 1 < nq) issue_dpt(s2);
             }
             umma_commit(bar(L::kAccFull));
             umma_commit(bar(L::kDrain));
@@ -396,7 +411,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait(bar(L::kDrain), 0, drain);
         }
     } else {
-        // ===================== recompute P^T, dS^T (one thread per key) =====================
+        // ===================== recompute P^T, dS^T (one thread per key, 64 queries) =====================
+        const int g = warp >> 2;            // column half: queries [64g, 64g+64) of each tile
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const int key = kv0 + row;
@@ -408,63 +424,65 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         for (int jj = 0; jj < nq; ++jj) {
             const int s = jj & 1;
-            const int q0 = (j_begin + jj) * kBQ;
-            const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256;
-            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2) -> tensor memory (16-bit)
+            const int qg = (j_begin + jj) * kBQ + 64 * g;     // first query of this thread's half
+            const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256 + 64 * g;
+            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2), kept in registers
             {
                 const bool got = mbar_wait(bar(L::kSFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
-            const bool diag = CAUSAL && (key > q0 + p.causal_off);   // some column masked
-            float pr[128];
+            const bool diag = CAUSAL && (key > qg + p.causal_off);   // some column masked
+            float pr[64];
+            {
+                uint32_t sv[64];
+                tmem_ld32dp_x64_wait(tl + L::kColS + 64 * g, sv);
+                const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32];
-                tmem_ld32dp_x32_wait(tl + L::kColS + c * 32, sv);
-                const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf + c * 32);
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
+                for (int e4 = 0; e4 < 16; ++e4) {
                     const float4 lv = l4[e4];
                     const float la[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int e = 4 * e4 + u;
                         float x = fmaf(__uint_as_float(sv[e]), qk, b2 - la[u]);
-                        if (diag && key > q0 + c * 32 + e + p.causal_off) x = neg_inf();
-                        pr[c * 32 + e] = ex2_approx(x);
+                        if (diag && key > qg + e + p.causal_off) x = neg_inf();
+                        pr[e] = ex2_approx(x);
                     }
                 }
-                uint32_t pp[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) pp[e] = pack2<BF16>(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
-                tmem_st32dp_x16(tl + L::kColP + c * 16, pp);
             }
-            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(L::kPTFull));
-            // ---- phase 2: dS^T = P^T (dP^T - D) -> tensor memory (16-bit)
+            mbar_arrive(bar(L::kPTFull));   // S^T loaded: its columns may be overwritten
+            // ---- phase 2: dS^T = P^T (dP^T - D); P^T and dS^T (16-bit) -> the
+            // dP^T columns this thread has just read
             {
                 const bool got = mbar_wait(bar(L::kDPFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
+            {
+                // two halves of 32 columns keep the live registers low; every
+                // dP^T column of this thread is loaded before anything is stored
+                uint32_t dpv[64];
+                tmem_ld32dp_x64_wait(tl + L::kColDP + 64 * g, dpv);
+                const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t dpv[32];
-                tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
-                const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128 + c * 32);
-                uint32_t dd[16];
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pp[16], dd[16];
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 dv = d4[e4];
-                    const int e = c * 32 + 4 * e4;
-                    dd[2 * e4] = pack2<BF16>(pr[e] * (__uint_as_float(dpv[4 * e4]) - dv.x),
-                                             pr[e + 1] * (__uint_as_float(dpv[4 * e4 + 1]) - dv.y));
-                    dd[2 * e4 + 1] = pack2<BF16>(pr[e + 2] * (__uint_as_float(dpv[4 * e4 + 2]) - dv.z),
-                                                 pr[e + 3] * (__uint_as_float(dpv[4 * e4 + 3]) - dv.w));
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 dv = d4[8 * h + e4];
+                        const int e = 32 * h + 4 * e4;
+                        pp[2 * e4] = pack2<BF16>(pr[e], pr[e + 1]);
+                        pp[2 * e4 + 1] = pack2<BF16>(pr[e + 2], pr[e + 3]);
+                        dd[2 * e4] = pack2<BF16>(pr[e] * (__uint_as_float(dpv[e]) - dv.x),
+                                                 pr[e + 1] * (__uint_as_float(dpv[e + 1]) - dv.y));
+                        dd[2 * e4 + 1] = pack2<BF16>(pr[e + 2] * (__uint_as_float(dpv[e + 2]) - dv.z),
+                                                     pr[e + 3] * (__uint_as_float(dpv[e + 3]) - dv.w));
+                    }
+                    tmem_st32dp_x16(tl + L::kColP + 64 * g + 16 * h, pp);
+                    tmem_st32dp_x16(tl + L::kColDS + 64 * g + 16 * h, dd);
                 }
-                tmem_st32dp_x16(tl + L::kColDS + c * 16, dd);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -478,8 +496,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tc_fence_after();
         }
         if (ok) {
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {       // 0: dV, 1: dK
+            {
+                const int which = g;                        // warpgroup 0: dV, 1: dK
                 const uint32_t col = which ? L::kColDK : L::kColDV;
                 const float mul = which ? p.scale : 1.f;
                 uint8_t *stage = smem + (which ? L::kK : L::kV);
@@ -504,8 +522,10 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int row0 = kv0 + wq * 32;
             if (lane == 0 && row0 < p.Nk) {
                 for (int c = 0; c < D / 64; ++c) {
-                    tma_store_3d(&tm_dv, sbase + L::kV + c * L::kChunkBytes + wq * 32 * 128, c * 64, row0, bh);
-                    tma_store_3d(&tm_dk, sbase + L::kK + c * L::kChunkBytes + wq * 32 * 128, c * 64, row0, bh);
+                    if (g == 0)
+                        tma_store_3d(&tm_dv, sbase + L::kV + c * L::kChunkBytes + wq * 32 * 128, c * 64, row0, bh);
+                    else
+                        tma_store_3d(&tm_dk, sbase + L::kK + c * L::kChunkBytes + wq * 32 * 128, c * 64, row0, bh);
                 }
                 tma_store_commit();
                 tma_store_wait_all();
@@ -583,7 +603,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(bar(L::kSFull + 0), 1);
         mbar_init(bar(L::kSFull + 1), 1);
         mbar_init(bar(L::kDPFull), 1);
-        mbar_init(bar(L::kDSFull), 128);
+        mbar_init(bar(L::kDSFull), kRecompute);
         mbar_init(bar(L::kOFull), 1);
         mbar_init(bar(L::kDrain), 1);
         fence_mbar_init();
@@ -734,7 +754,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t a = tmem + ((j & 1) ? L::kColS1 : L::kColS0);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDQ, a + kk * 8, smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024),
+                    umma_f16_ts(tmem + L::kColDQ, a + (kk >> 2) * 64 + (kk & 3) * 8,
+                                smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024),
                                 idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
                 if (j + 3 < n) umma_commit(bar(L::kKEmpty + j % L::kKStages));
                 if (j + 1 < n) {
@@ -759,7 +780,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_wait(bar(L::kDrain), 0, drain);
         }
     } else {
-        // ===================== recompute P, dS (one thread per query row) =====================
+        // ===================== recompute P, dS (one thread per query row, 64 keys) =====================
+        const int g = warp >> 2;            // column half: keys [64g, 64g+64) of each tile
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const int q = q0 + row;
@@ -775,7 +797,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int lim = CAUSAL ? min(q + p.causal_off, p.Nk - 1) : p.Nk - 1;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
-            const int kv0 = j * kBK;
+            const int kg = j * kBK + 64 * g;                  // first key of this thread's half
             const uint32_t tS = tl + ((j & 1) ? L::kColS1 : L::kColS0);
             {
                 const bool got = mbar_wait(bar(L::kSFull + (j & 1)), (j >> 1) & 1, wctx);
@@ -783,22 +805,22 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             tc_fence_after();
             // ---- P = 2^(S qk + bias - LSE_2), kept in registers
-            float pr[128];
-            const float *bs = reinterpret_cast<const float *>(smem + L::kBias) + (j % L::kKStages) * 128;
-            const bool edge = kv0 + kBK - 1 > lim;
+            float pr[64];
+            {
+                uint32_t sv[64];
+                tmem_ld32dp_x64_wait(tS + 64 * g, sv);
+                const float *bs = reinterpret_cast<const float *>(smem + L::kBias) +
+                                  (j % L::kKStages) * 128 + 64 * g;
+                const bool edge = kg + 63 > lim;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32];
-                tmem_ld32dp_x32_wait(tS + c * 32, sv);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < 64; ++e) {
                     float x;
                     if constexpr (HAS_BIAS)
-                        x = fmaf(__uint_as_float(sv[e]), qk, bs[c * 32 + e] - lse2);
+                        x = fmaf(__uint_as_float(sv[e]), qk, bs[e] - lse2);
                     else
                         x = fmaf(__uint_as_float(sv[e]), qk, -lse2);
-                    if (edge && kv0 + c * 32 + e > lim) x = neg_inf();
-                    pr[c * 32 + e] = ex2_approx(x);
+                    if (edge && kg + e > lim) x = neg_inf();
+                    pr[e] = ex2_approx(x);
                 }
             }
             // ---- dS = P (dP - D) -> tensor memory (16-bit), over the S columns
@@ -807,22 +829,22 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
+            {
+                uint32_t dpv[64];
+                tmem_ld32dp_x64_wait(tl + L::kColDP + 64 * g, dpv);
+                uint32_t dd[32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t dpv[32];
-                tmem_ld32dp_x32_wait(tl + L::kColDP + c * 32, dpv);
-                uint32_t dd[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    dd[e] = pack2<BF16>(pr[c * 32 + 2 * e] * (__uint_as_float(dpv[2 * e]) - di),
-                                        pr[c * 32 + 2 * e + 1] * (__uint_as_float(dpv[2 * e + 1]) - di));
-                tmem_st32dp_x16(tS + c * 16, dd);
+                for (int e = 0; e < 32; ++e)
+                    dd[e] = pack2<BF16>(pr[2 * e] * (__uint_as_float(dpv[2 * e]) - di),
+                                        pr[2 * e + 1] * (__uint_as_float(dpv[2 * e + 1]) - di));
+                tmem_st32dp_x32(tS + 64 * g, dd);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::kDSFull));
         }
-        // ---- epilogue: dQ = scale * acc, 16-bit, staged in the (idle) Q buffer
+        // ---- epilogue (warpgroup 0): dQ = scale * acc, 16-bit, staged in the (idle) Q buffer
+        if (g != 0) ok = false;
         if (ok && n > 0) {
             const bool got = mbar_wait(bar(L::kOFull), 0, wctx);
             ok = __all_sync(0xffffffffu, got);
