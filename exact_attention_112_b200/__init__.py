@@ -22,7 +22,8 @@ import threading
 __all__ = [
     "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
-    "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes",
+    "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_noalloc",
+    "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "attention_forward", "attention_backward",
 ]
@@ -65,6 +66,9 @@ def lib() -> ctypes.CDLL:
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
                                  vp, vp, sz, vp]
             L.fa_bwd.restype = i
+            L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f,
+                                         i, vp, vp]
+            L.fa_bwd_noalloc.restype = i
             L.fa_status_string.argtypes = [i]
             L.fa_status_string.restype = ctypes.c_char_p
             L.fa_device_status.argtypes = [vp]
@@ -140,6 +144,24 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, causal=False, scale=None,
                       _dtype_code(q), _ptr(key_bias), _ptr(workspace), nbytes,
                       _stream_ptr(stream))
     _check(st, "fa_bwd")
+
+
+FA_BWD_NOALLOC_MAX_ROWS = 1048576
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, causal=False, scale=None, key_bias=None,
+                   stream=None):
+    """Backward without a workspace, for callers that cannot allocate device
+    memory (the scratch is a fixed array inside libfa.so; B*H*Nq must not
+    exceed FA_BWD_NOALLOC_MAX_ROWS).  See include/fa.h."""
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)),
+                              float(scale), _dtype_code(q), _ptr(key_bias), _stream_ptr(stream))
+    _check(st, "fa_bwd_noalloc")
 
 
 def fa_device_status(stream=None) -> int:

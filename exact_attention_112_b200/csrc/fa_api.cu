@@ -282,3 +282,55 @@ extern "C" int fa_debug_wait_timeout(unsigned timeout_us, void *stream) {
     fa::note_launch();
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
+
+// ---- allocation-free backward ----------------------------------------------
+// Some callers may not allocate device memory at all once they are running:
+// services that reserve their whole memory budget at start-up and forbid
+// allocation on the request path, plugin hosts that hand a library only its
+// input and output buffers, and latency-critical paths where an allocation's
+// cost or possible failure is not acceptable.  fa_bwd_noalloc serves them with
+// a fixed scratch array compiled into the library instead of a workspace
+// argument.  The array is file-scope device memory: every GPU that loads the
+// library holds it until the process exits.
+namespace {
+constexpr size_t kNoAllocMaxRows = FA_BWD_NOALLOC_MAX_ROWS;
+// D_i of every query row (4 bytes per row) plus the 256 bytes of alignment
+// slack that fa_bwd_workspace_bytes() counts.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxRows + 64];
+std::mutex g_noalloc_mu;
+float *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name only stands in for the symbol; the address a kernel may
+// use has to be asked of the runtime, once per device.
+int noalloc_scratch(int dev, float **out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+            return FA_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return FA_OK;
+}
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                              const float *lse, const void *dO, void *dq, void *dk, void *dv, int B,
+                              int H, int Nq, int Nk, int D, int causal, float scale, int dtype,
+                              const float *key_bias, void *stream) {
+    // Too many query rows for the fixed scratch: refuse before touching the GPU.
+    if (B >= 1 && H >= 1 && Nq >= 0 &&
+        static_cast<long long>(B) * H * Nq > static_cast<long long>(kNoAllocMaxRows))
+        return FA_ERR_WORKSPACE;
+    int dev;
+    int st = current_device(&dev);
+    if (st != FA_OK) return st;
+    float *scratch = nullptr;
+    if ((st = noalloc_scratch(dev, &scratch)) != FA_OK) return st;
+    // Every scratch entry the kernels read is written earlier in the same call
+    // (the row-term pre-pass covers every query row), so nothing needs clearing.
+    return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, causal, scale, dtype, key_bias,
+                  scratch, sizeof(g_noalloc_scratch), stream);
+}

@@ -98,6 +98,37 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            int dtype, const float *key_bias, void *workspace,
            size_t workspace_bytes, void *stream);
 
+/*
+ * Largest B * H * Nq that fa_bwd_noalloc() accepts.
+ */
+#define FA_BWD_NOALLOC_MAX_ROWS 1048576
+
+/*
+ * fa_bwd() for callers that cannot allocate device memory: services that
+ * reserve their whole memory budget at start-up and allow no allocation while
+ * serving, plugin hosts that give a library only its input and output
+ * buffers, and latency-critical paths that cannot afford an allocation or its
+ * failure.  No page describes this entry point; it exists for those callers.
+ *
+ * Arguments, layouts and results are those of fa_bwd() without the workspace:
+ * the per-row scratch lives in a fixed array compiled into the library
+ * (4 * FA_BWD_NOALLOC_MAX_ROWS bytes plus 256, held on every GPU that loads the
+ * library until the process exits).  Nothing is allocated by this call.
+ *   - B * H * Nq > FA_BWD_NOALLOC_MAX_ROWS returns FA_ERR_WORKSPACE before any
+ *     GPU work.
+ *   - The first call on a device asks the CUDA runtime for the array's device
+ *     address (cudaGetSymbolAddress); make that first call before any stream
+ *     capture begins.
+ *   - All calls share the one array and every call writes the parts it reads,
+ *     so what an earlier call left there does not matter; but two calls whose
+ *     work overlaps on the GPU (different streams without ordering between
+ *     them) race on it and may return wrong gradients.
+ */
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                   const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                   int B, int H, int Nq, int Nk, int D, int causal, float scale,
+                   int dtype, const float *key_bias, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);
 
