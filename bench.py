@@ -90,6 +90,53 @@ WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention back
                    "sweep": "sequence-sweep attention"}
 
 
+# Algorithmic FLOPs of one launch of each kernel, as multiples of the forward's
+# 4*B*H*Nq*Nk*D (halved for causal).  The backward's five tile products
+# (S, dP, dV, dK, dQ) are split between the two recompute kernels: the dK/dV
+# kernel does S^T, dP^T, dV, dK (4 of 5 = 2.0x forward); the dQ kernel does dQ
+# (0.5x forward) plus a recomputation of S and dP that is not algorithmic work.
+KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5}
+# tile products each kernel executes, as multiples of the forward (2 products)
+KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5}
+
+
+def max_over_ranks(x, world, device=None):
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, step_flops, steps, t_max_ms):
+    """Whole-job TFLOP/s: every rank did `steps` steps of `step_flops`; the job
+    took as long as its slowest rank."""
+    return world * step_flops * steps / (t_max_ms * 1e-3) / 1e12
+
+
+def kernel_table(records, w):
+    """Per-kernel totals of fa_profile_read() records over the timed steps."""
+    from exact_attention_112_b200 import metrics
+    f1 = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    agg = {}
+    for name, ms in records:
+        a = agg.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += ms
+    total = sum(a[1] for a in agg.values()) or 1.0
+    out = {}
+    for name, (n, ms) in agg.items():
+        e = {"launches": n, "ms_per_launch": ms / n, "share": ms / total}
+        if name in KERNEL_FWD_MULTIPLE:
+            e["algorithmic_tflops"] = KERNEL_FWD_MULTIPLE[name] * f1 / (ms / n * 1e-3) / 1e12
+            e["executed_tflops"] = KERNEL_EXEC_MULTIPLE[name] * f1 / (ms / n * 1e-3) / 1e12
+        out[name] = e
+    return out
+
+
 def workload_name(w, passes):
     return (f"{WORKLOAD_TITLES.get(w['name'], w['name'])} {'+'.join(passes)}: B={w['B']} H={w['H']} "
             f"Nq={w['Nq']} Nk={w['Nk']} D={w['D']} "
@@ -313,11 +360,15 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     launches0 = fa.fa_launch_count()
+    fa.fa_profile_read()                   # drop anything recorded before
+    fa.fa_profile_enable(True)
     for s in range(args.steps):
         flush.zero_()                      # L2 flush outside the timed events
         step(evs[s])
     torch.cuda.synchronize(dev)
+    fa.fa_profile_enable(False)
     launches = fa.fa_launch_count() - launches0
+    kernels = kernel_table(fa.fa_profile_read(capacity=16 * args.steps + 64), w)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -329,15 +380,10 @@ def run_ours(args):
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if "bwd" in passes else []
     step_ms = [f + b for f, b in zip(fwd_ms, bwd_ms or [0.0] * len(fwd_ms))]
     t_local = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([t_local], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    else:
-        t_max = t_local
+    t_max = max_over_ranks(t_local, world, dev)
     fl = flops_of(w, passes)
     step_flops = sum(fl.values())
-    value = world * step_flops * args.steps / (t_max * 1e-3) / 1e12
+    value = weak_scaling_value(world, step_flops, args.steps, t_max)
 
     # ---- end to end through the public binding, host buffers
     host = {x: inp[x].pin_memory() for x in ("q", "k", "v")}
@@ -375,26 +421,21 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * step_flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = weak_scaling_value(world, step_flops, args.e2e_steps, e2e_ms)
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant kernel (largest share of the timed device time)
     peaks, peak_kind = load_peaks()
     kern_ms = {"fwd": statistics.mean(fwd_ms)}
     if bwd_ms:
         kern_ms["bwd"] = statistics.mean(bwd_ms)
-    dom = max(kern_ms, key=kern_ms.get)
     peak = float(peaks["bf16_tflops"])
-    achieved = fl[dom] / (kern_ms[dom] * 1e-3) / 1e12
-    traffic = load_traffic(dom, w)
+    dom = max((k for k in kernels if k in KERNEL_FWD_MULTIPLE), key=lambda k: kernels[k]["share"])
+    achieved = kernels[dom]["algorithmic_tflops"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-            "frac": achieved / peak, "traffic": traffic, "kernel": f"fa_{dom}",
-            "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
-            else "fallback 1.59 PFLOP/s"}
+            "frac": achieved / peak, "traffic": load_traffic(dom, w), "kernel": dom,
+            "peak_source": (f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                            else "fallback 1.59 PFLOP/s")}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -413,6 +454,7 @@ def run_ours(args):
         "per_pass": {p: {"ms": kern_ms[p], "tflops": fl[p] / (kern_ms[p] * 1e-3) / 1e12,
                          "frac_of_peak": fl[p] / (kern_ms[p] * 1e-3) / 1e12 / peak}
                      for p in kern_ms},
+        "kernels": kernels,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, passes)
@@ -423,7 +465,7 @@ def run_ours(args):
     return 0
 
 
-def load_traffic(kind, w):
+def load_traffic(kernel, w):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary (profiles/), or None if none matches the current kernel build."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -431,7 +473,7 @@ def load_traffic(kind, w):
         return None
     try:
         d = json.load(open(path))
-        ent = d.get(f"fa_{kind}:{w['name']}")
+        ent = d.get(f"{kernel}:{w['name']}")
         if ent and ent.get("kernel_rev") == kernel_rev():
             return ent["bytes_per_launch"]
     except (OSError, ValueError):

@@ -25,6 +25,7 @@ __all__ = [
     "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_noalloc",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
+    "fa_profile_enable", "fa_profile_read",
     "attention_forward", "attention_backward",
 ]
 
@@ -73,6 +74,12 @@ def lib() -> ctypes.CDLL:
             L.fa_status_string.restype = ctypes.c_char_p
             L.fa_device_status.argtypes = [vp]
             L.fa_device_status.restype = i
+            L.fa_profile_enable.argtypes = [i]
+            L.fa_profile_enable.restype = i
+            L.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float),
+                                          ctypes.POINTER(ctypes.c_char_p), i,
+                                          ctypes.POINTER(ctypes.c_int)]
+            L.fa_profile_read.restype = i
             L.fa_launch_count.argtypes = []
             L.fa_launch_count.restype = ctypes.c_ulonglong
             L.fa_debug_wait_timeout.argtypes = [ctypes.c_uint, vp]
@@ -166,6 +173,20 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, causal=False, scale=None, ke
 
 def fa_device_status(stream=None) -> int:
     return int(lib().fa_device_status(_stream_ptr(stream)))
+
+
+def fa_profile_enable(on: bool = True) -> None:
+    _check(lib().fa_profile_enable(int(bool(on))), "fa_profile_enable")
+
+
+def fa_profile_read(capacity: int = 4096):
+    """[(kernel name, milliseconds), ...] of the launches recorded since the
+    last read on this thread (see fa_profile_enable)."""
+    ms = (ctypes.c_float * capacity)()
+    names = (ctypes.c_char_p * capacity)()
+    n = ctypes.c_int(0)
+    _check(lib().fa_profile_read(ms, names, capacity, ctypes.byref(n)), "fa_profile_read")
+    return [(names[i].decode(), float(ms[i])) for i in range(n.value)]
 
 
 def fa_launch_count() -> int:

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "fa.h"
 #include "fa_internal.h"
@@ -104,13 +105,63 @@ int check_common(int B, int H, int Nq, int Nk, int D, int causal, float scale, i
 
 std::atomic<unsigned long long> g_launches{0};
 
+struct ProfRecord {
+    const char *name;
+    cudaEvent_t start, stop;
+};
+thread_local bool t_prof_on = false;
+thread_local std::vector<ProfRecord> t_prof;
+
 }  // namespace
 
 void fa::note_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+void fa::prof_begin(cudaStream_t stream, const char *name) {
+    if (!t_prof_on) return;
+    ProfRecord r{name, nullptr, nullptr};
+    if (cudaEventCreate(&r.start) != cudaSuccess) return;
+    if (cudaEventCreate(&r.stop) != cudaSuccess) {
+        cudaEventDestroy(r.start);
+        return;
+    }
+    cudaEventRecord(r.start, stream);
+    t_prof.push_back(r);
+}
+
+void fa::prof_end(cudaStream_t stream) {
+    if (!t_prof_on || t_prof.empty()) return;
+    cudaEventRecord(t_prof.back().stop, stream);
+}
+
 extern "C" {
 
 unsigned long long fa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int fa_profile_enable(int on) {
+    t_prof_on = on != 0;
+    return FA_OK;
+}
+
+int fa_profile_read(float *ms, const char **names, int capacity, int *count) {
+    if (capacity < 0 || (capacity > 0 && !ms) || !count) return FA_ERR_INVALID_ARG;
+    int n = 0;
+    int st = FA_OK;
+    for (ProfRecord &r : t_prof) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            st = FA_ERR_CUDA;
+        if (n < capacity) {
+            ms[n] = t;
+            if (names) names[n] = r.name;
+            ++n;
+        }
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+    }
+    t_prof.clear();
+    *count = n;
+    return st;
+}
 
 const char *fa_status_string(int status) {
     switch (status) {
@@ -277,8 +328,10 @@ extern "C" int fa_debug_wait_timeout(unsigned timeout_us, void *stream) {
     int *err = nullptr;
     if ((st = device_setup(dev, &err)) != FA_OK) return st;
     if (timeout_us == 0 || timeout_us > 10000000u) return FA_ERR_INVALID_ARG;
+    fa::prof_begin(static_cast<cudaStream_t>(stream), "fa_wait_timeout_kernel");
     fa_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         err, static_cast<unsigned long long>(timeout_us) * 1000ull);
+    fa::prof_end(static_cast<cudaStream_t>(stream));
     fa::note_launch();
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

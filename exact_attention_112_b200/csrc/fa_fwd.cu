@@ -473,7 +473,9 @@ cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, cudaStream
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H;
+    prof_begin(stream, "fa_fwd_kernel");
     kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    prof_end(stream);
     note_launch();
     return cudaGetLastError();
 }
@@ -498,10 +500,12 @@ cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool 
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>(std::min<size_t>((n_rows + 255) / 256, 4096));
     if (grid == 0) return cudaSuccess;
+    prof_begin(stream, "fa_fwd_empty_kernel");
     if (bf16)
         fa_fwd_empty_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(o), lse, n_rows, D);
     else
         fa_fwd_empty_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<__half *>(o), lse, n_rows, D);
+    prof_end(stream);
     note_launch();
     return cudaGetLastError();
 }

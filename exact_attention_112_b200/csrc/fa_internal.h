@@ -49,6 +49,11 @@ cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool 
 // Counts every kernel launch made by the library (fa_launch_count()).
 void note_launch(unsigned n = 1);
 
+// Per-kernel timing aid (fa_profile_enable / fa_profile_read): when enabled on
+// the calling host thread, each launch is bracketed by two events on its stream.
+void prof_begin(cudaStream_t stream, const char *name);
+void prof_end(cudaStream_t stream);
+
 cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                        bool has_bias, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,

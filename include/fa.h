@@ -146,6 +146,18 @@ int fa_device_status(void *stream);
 unsigned long long fa_launch_count(void);
 
 /*
+ * Per-kernel device timing, a measurement aid.  While enabled on the calling
+ * host thread, every kernel the library launches from that thread is
+ * bracketed by two CUDA events recorded on its stream.  fa_profile_read()
+ * waits for those events, writes each kernel's elapsed milliseconds (launch
+ * order) into ms[0 .. *count) and, if names is not NULL, a static kernel name
+ * into names[i]; then it forgets them.  Records beyond `capacity` are dropped.
+ * Profiling stays enabled until fa_profile_enable(0).
+ */
+int fa_profile_enable(int on);
+int fa_profile_read(float *ms, const char **names, int capacity, int *count);
+
+/*
  * Self-test of the bounded-wait mechanism: launches one block that waits on a
  * barrier nothing will ever complete, with a limit of `timeout_us`
  * microseconds; the kernel must give up, latch FA_ERR_DEVICE_TIMEOUT and
