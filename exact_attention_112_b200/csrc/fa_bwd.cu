@@ -896,7 +896,9 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
+        prof_begin(stream, "fa_bwd_dkdv_kernel");
         kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, p);
+        prof_end(stream);
         note_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -906,7 +908,9 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
+        prof_begin(stream, "fa_bwd_dq_kernel");
         kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dq, p);
+        prof_end(stream);
         note_launch();
         return cudaGetLastError();
     }
@@ -919,8 +923,10 @@ cudaError_t launch_bwd_d(const BwdTensorMaps &tm, const BwdParams &p, bool causa
     {
         const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
         const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+        prof_begin(s, "fa_bwd_pre_kernel");
         fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
                                                          static_cast<const uint16_t *>(p.dO), p.Di, rows);
+        prof_end(s);
         note_launch();
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
