@@ -438,17 +438,27 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 uint32_t sv[64];
                 tmem_ld32dp_x64_wait(tl + L::kColS + 64 * g, sv);
                 const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf);
+                const float2 qk2 = make_float2(qk, qk);
+                const float2 b22 = make_float2(b2, b2);
 #pragma unroll
                 for (int e4 = 0; e4 < 16; ++e4) {
                     const float4 lv = l4[e4];
-                    const float la[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = 4 * e4 + u;
-                        float x = fmaf(__uint_as_float(sv[e]), qk, b2 - la[u]);
-                        if (diag && key > qg + e + p.causal_off) x = neg_inf();
-                        pr[e] = ex2_approx(x);
+                    // x = s qk + (bias - LSE_2), two columns per instruction
+                    const float2 c01 = __fadd2_rn(b22, make_float2(-lv.x, -lv.y));
+                    const float2 c23 = __fadd2_rn(b22, make_float2(-lv.z, -lv.w));
+                    float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4]), __uint_as_float(sv[4 * e4 + 1])), qk2, c01);
+                    float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])), qk2, c23);
+                    if (diag) {
+                        const int e = 4 * e4;
+                        if (key > qg + e + p.causal_off) x01.x = neg_inf();
+                        if (key > qg + e + 1 + p.causal_off) x01.y = neg_inf();
+                        if (key > qg + e + 2 + p.causal_off) x23.x = neg_inf();
+                        if (key > qg + e + 3 + p.causal_off) x23.y = neg_inf();
                     }
+                    pr[4 * e4] = ex2_approx(x01.x);
+                    pr[4 * e4 + 1] = ex2_approx(x01.y);
+                    pr[4 * e4 + 2] = ex2_approx(x23.x);
+                    pr[4 * e4 + 3] = ex2_approx(x23.y);
                 }
             }
             tc_fence_before();
@@ -475,10 +485,14 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         const int e = 32 * h + 4 * e4;
                         pp[2 * e4] = pack2<BF16>(pr[e], pr[e + 1]);
                         pp[2 * e4 + 1] = pack2<BF16>(pr[e + 2], pr[e + 3]);
-                        dd[2 * e4] = pack2<BF16>(pr[e] * (__uint_as_float(dpv[e]) - dv.x),
-                                                 pr[e + 1] * (__uint_as_float(dpv[e + 1]) - dv.y));
-                        dd[2 * e4 + 1] = pack2<BF16>(pr[e + 2] * (__uint_as_float(dpv[e + 2]) - dv.z),
-                                                     pr[e + 3] * (__uint_as_float(dpv[e + 3]) - dv.w));
+                        const float2 d01 = __fmul2_rn(make_float2(pr[e], pr[e + 1]),
+                                                      __fadd2_rn(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                                                 make_float2(-dv.x, -dv.y)));
+                        const float2 d23 = __fmul2_rn(make_float2(pr[e + 2], pr[e + 3]),
+                                                      __fadd2_rn(make_float2(__uint_as_float(dpv[e + 2]), __uint_as_float(dpv[e + 3])),
+                                                                 make_float2(-dv.z, -dv.w)));
+                        dd[2 * e4] = pack2<BF16>(d01.x, d01.y);
+                        dd[2 * e4 + 1] = pack2<BF16>(d23.x, d23.y);
                     }
                     tmem_st32dp_x16(tl + L::kColP + 64 * g + 16 * h, pp);
                     tmem_st32dp_x16(tl + L::kColDS + 64 * g + 16 * h, dd);
@@ -812,15 +826,22 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const float *bs = reinterpret_cast<const float *>(smem + L::kBias) +
                                   (j % L::kKStages) * 128 + 64 * g;
                 const bool edge = kg + 63 > lim;
+                const float2 qk2 = make_float2(qk, qk);
+                const float2 nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    float x;
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 sc = make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+                    float2 x;
                     if constexpr (HAS_BIAS)
-                        x = fmaf(__uint_as_float(sv[e]), qk, bs[e] - lse2);
+                        x = __ffma2_rn(sc, qk2, __fadd2_rn(make_float2(bs[e], bs[e + 1]), nl2));
                     else
-                        x = fmaf(__uint_as_float(sv[e]), qk, -lse2);
-                    if (edge && kg + e > lim) x = neg_inf();
-                    pr[e] = ex2_approx(x);
+                        x = __ffma2_rn(sc, qk2, nl2);
+                    if (edge) {
+                        if (kg + e > lim) x.x = neg_inf();
+                        if (kg + e + 1 > lim) x.y = neg_inf();
+                    }
+                    pr[e] = ex2_approx(x.x);
+                    pr[e + 1] = ex2_approx(x.y);
                 }
             }
             // ---- dS = P (dP - D) -> tensor memory (16-bit), over the S columns
@@ -833,10 +854,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint32_t dpv[64];
                 tmem_ld32dp_x64_wait(tl + L::kColDP + 64 * g, dpv);
                 uint32_t dd[32];
+                const float2 nd2 = make_float2(-di, -di);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    dd[e] = pack2<BF16>(pr[2 * e] * (__uint_as_float(dpv[2 * e]) - di),
-                                        pr[2 * e + 1] * (__uint_as_float(dpv[2 * e + 1]) - di));
+                for (int e = 0; e < 32; ++e) {
+                    const float2 d = __fmul2_rn(make_float2(pr[2 * e], pr[2 * e + 1]),
+                                                __fadd2_rn(make_float2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), nd2));
+                    dd[e] = pack2<BF16>(d.x, d.y);
+                }
                 tmem_st32dp_x32(tS + 64 * g, dd);
             }
             tmem_wait_st();

@@ -39,8 +39,9 @@
 // Shared memory: Q_0, Q_1 (reused as O staging for the TMA store), K ring x2,
 // V ring x2, mbarriers.
 //
-// Warp roles (10 warps): 0-3 softmax of Q_0, 4-7 softmax of Q_1, 8 TMA
-// producer, 9 MMA issuer (also allocates tensor memory).
+// Warp roles (12 warps): 0-3 softmax of Q_0, 4-7 softmax of Q_1, 8 TMA
+// producer, 9 MMA issuer (also allocates tensor memory), 10-11 idle (they
+// only complete the third warpgroup for the register split).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -58,9 +59,14 @@ namespace {
 
 constexpr int kBM = 128;            // query rows per tensor-core tile
 constexpr int kBN = 128;            // keys per tile
-constexpr int kThreads = 320;       // 10 warps
+constexpr int kThreads = 384;       // 12 warps = three warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split (launch pool 168 x 384 = 64512): the two softmax warpgroups
+// take 192 each, the producer/MMA warpgroup (warps 8-11, 10-11 idle) 120:
+// 8*32*192 + 4*32*120 = 64512; per SMSP (192 + 192 + 120) * 32 = 16128 <= 16384.
+constexpr uint32_t kRegsSoftmax = 192;
+constexpr uint32_t kRegsOther = 120;
 constexpr int kStages = 2;
 constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -169,7 +175,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
-
+    // Register split: warpgroup 2 (producer, MMA, two idle warps) gives
+    // registers back, the softmax warpgroups take them.  Nobody asks for
+    // registers again afterwards, so the split cannot deadlock; every role ends
+    // in its own branch at the CTA barrier 1, and the MMA warp frees tensor
+    // memory after it.
+    if (warp >= 8) regs_release<kRegsOther>();
     if (warp == kProducerWarp) {
         // ===================== TMA producer =====================
         if (lane == 0 && n_kv > 0) {
@@ -210,6 +221,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
         }
+        named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
         // ===================== MMA issuer (one thread) =====================
         if (lane == 0 && n_kv > 0) {
@@ -282,8 +294,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             drain.abort_flag = &zero;
             mbar_wait(bar(L::kDrain), 0, drain);
         }
-    } else {
+        named_bar_sync(1, kThreads);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    } else if (warp < 8) {
         // ===================== softmax warpgroups =====================
+        regs_alloc<kRegsSoftmax>();
         const int i = warp >> 2;            // which Q tile
         const int wq = warp & 3;            // lane quarter of tensor memory
         const int row = wq * 32 + lane;     // row within the tile (= TMEM lane)
@@ -351,45 +368,53 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
             if constexpr (!HAS_BIAS) m_tile *= qk;   // qk > 0: max commutes with scaling
             const bool need = m_tile > m_ref + kTau;
-            if (__any_sync(0xffffffffu, need)) {
+            // warp-uniform: if any row of the warp moves its reference maximum,
+            // the warp rescales its O rows (after P is formed, below)
+            const bool rescale = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (rescale) {
                 const float m_new = need ? m_tile : m_ref;
-                const float alpha = (m_ref == neg_inf()) ? 0.f : ex2_approx(m_ref - m_new);
+                alpha = (m_ref == neg_inf()) ? 0.f : ex2_approx(m_ref - m_new);
                 l *= alpha;
-                if (j > 0) {
-                    // O_i row *= alpha (O is stable: the MMA that produced this
-                    // S tile was issued after the previous P.V and its commit
-                    // covers it).
-#pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t orr[32];
-                        tmem_ld32dp_x32_wait(tO + cc * 32, orr);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32dp_x32(tO + cc * 32, orr);
-                    }
-                }
                 m_ref = m_new;
             }
             const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
-            uint32_t pk[64];
-            float l0 = 0.f, l1 = 0.f;
+            // p = 2^(x - m), two columns per paired-fp32 instruction.  P goes
+            // back into the S columns in two halves (every S value is already
+            // in registers), which keeps the live registers low.
+            float2 lsum = make_float2(0.f, 0.f);
+            const float2 neg_m2 = make_float2(-m_use, -m_use);
+            const float2 qk2 = make_float2(qk, qk);
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                float p0, p1;
-                if constexpr (HAS_BIAS) {
-                    p0 = ex2_approx(x[c] - m_use);
-                    p1 = ex2_approx(x[c + 1] - m_use);
-                } else {
-                    p0 = ex2_approx(fmaf(x[c], qk, -m_use));
-                    p1 = ex2_approx(fmaf(x[c + 1], qk, -m_use));
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c2 = 0; c2 < 32; ++c2) {
+                    const int c = 64 * h + 2 * c2;
+                    const float2 xc = make_float2(x[c], x[c + 1]);
+                    const float2 a = HAS_BIAS ? __fadd2_rn(xc, neg_m2) : __ffma2_rn(xc, qk2, neg_m2);
+                    const float2 pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                    lsum = __fadd2_rn(lsum, pp);
+                    pk[c2] = pack2<BF16>(pp.x, pp.y);
                 }
-                l0 += p0;
-                l1 += p1;
-                pk[c >> 1] = pack2<BF16>(p0, p1);
+                tmem_st32dp_x32(tS + 32 * h, pk);
             }
+            const float l0 = lsum.x, l1 = lsum.y;
             l += l0 + l1;
-            tmem_st32dp_x64(tS, pk);
+            if (rescale && j > 0) {
+                // O_i row *= alpha.  O is stable: the MMA that produced this S
+                // tile was issued after the previous P.V and its commit covers
+                // it; the next P.V waits for the arrive below.
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t orr[32];
+                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    tmem_st32dp_x32(tO + cc * 32, orr);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::kPFull + i));
@@ -446,13 +471,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         tc_fence_before();
-    }
-
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, L::kTmemCols);
+        named_bar_sync(1, kThreads);
+    } else {
+        named_bar_sync(1, kThreads);   // idle warps 10, 11
     }
 }
 

@@ -70,7 +70,7 @@ struct WaitCtx {
 // Wait until the phase with the given parity of `bar` has completed.  Returns
 // false if the limit expires or another role of this CTA has aborted; the
 // first to give up latches kErrDeviceTimeout in the error word.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx &w) {
+static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx &w) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -139,6 +139,18 @@ __device__ __forceinline__ void tma_store_wait_all() {
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the same
+// instruction).  The CTA's pool is what it was launched with; a warpgroup that
+// asks for more waits until others have released enough.
+template <uint32_t N>
+__device__ __forceinline__ void regs_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_release() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
