@@ -39,9 +39,12 @@
 //                            (16-bit pairs) overwrites the first 32 of each
 //                            warpgroup's 64 columns
 //   cols [256,384)    dP (fp32),   cols [384,384+D) dQ accumulator
-// Warp roles (10 warps): 0-7 recompute/gradient (one thread per tile row and
+// Warp roles (12 warps): 0-7 recompute/gradient (one thread per tile row and
 // half of the tile's columns: warpgroup g owns columns [64g, 64g+64)), 8 TMA
-// producer, 9 MMA issuer.
+// producer, 9 MMA issuer, 10-11 idle (they complete the third warpgroup for
+// the register split).  Every role ends at CTA barrier 1 in its own branch and
+// no warp asks for registers after giving them up, so the split cannot
+// deadlock.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -58,10 +61,14 @@ namespace {
 
 constexpr int kBK = 128;          // keys per tile
 constexpr int kBQ = 128;          // queries per tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;     // three warpgroups
 constexpr int kRecompute = 256;   // two warpgroups, each owning 64 of a tile's 128 columns
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split (launch pool 168 x 384 = 64512): recompute warpgroups 192,
+// warpgroup 2 (producer, MMA, two idle warps) 120; per SMSP (192+192+120)*32 = 16128.
+constexpr uint32_t kRegsRecompute = 192;
+constexpr uint32_t kRegsOther = 120;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -281,6 +288,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
 
+    if (warp >= 8) regs_release<kRegsOther>();
     if (warp == kProducerWarp) {
         // ===================== producer =====================
         const float *lse_bh = p.lse + static_cast<size_t>(bh) * p.Nq;
@@ -338,6 +346,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int jj = (issued > 2 ? issued - 2 : 0); jj < issued; ++jj)
                 mbar_wait(bar(L::kQFull + (jj & 1)), (jj >> 1) & 1, drain);
         }
+        named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
         // ===================== MMA issuer =====================
         if (lane == 0) {
@@ -410,8 +419,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             drain.abort_flag = &zero;
             mbar_wait(bar(L::kDrain), 0, drain);
         }
-    } else {
+        named_bar_sync(1, kThreads);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    } else if (warp < 8) {
         // ===================== recompute P^T, dS^T (one thread per key, 64 queries) =====================
+        regs_alloc<kRegsRecompute>();
         const int g = warp >> 2;            // column half: queries [64g, 64g+64) of each tile
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
@@ -546,13 +560,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
         }
         tc_fence_before();
-    }
-
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, L::kTmemCols);
+        named_bar_sync(1, kThreads);
+    } else {
+        named_bar_sync(1, kThreads);   // idle warps 10, 11
     }
 }
 
@@ -635,6 +645,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{p.timeout_ns, p.err, abort_flag};
 
+    if (warp >= 8) regs_release<kRegsOther>();
     if (warp == kProducerWarp) {
         // ===================== producer =====================
         const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(bh / p.H) * p.Nk : nullptr;
@@ -715,6 +726,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int j = (v_issued > 2 ? v_issued - 2 : 0); j < v_issued; ++j)
                 mbar_wait(bar(L::kVFull + j % L::kVStages), (j / L::kVStages) & 1, drain);
         }
+        named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
         // ===================== MMA issuer =====================
         if (lane == 0 && n > 0) {
@@ -793,8 +805,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             drain.abort_flag = &zero;
             mbar_wait(bar(L::kDrain), 0, drain);
         }
-    } else {
+        named_bar_sync(1, kThreads);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    } else if (warp < 8) {
         // ===================== recompute P, dS (one thread per query row, 64 keys) =====================
+        regs_alloc<kRegsRecompute>();
         const int g = warp >> 2;            // column half: keys [64g, 64g+64) of each tile
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
@@ -902,13 +919,9 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         tc_fence_before();
-    }
-
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, L::kTmemCols);
+        named_bar_sync(1, kThreads);
+    } else {
+        named_bar_sync(1, kThreads);   // idle warps 10, 11
     }
 }
 
