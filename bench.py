@@ -95,9 +95,13 @@ WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention back
 # (S, dP, dV, dK, dQ) are split between the two recompute kernels: the dK/dV
 # kernel does S^T, dP^T, dV, dK (4 of 5 = 2.0x forward); the dQ kernel does dQ
 # (0.5x forward) plus a recomputation of S and dP that is not algorithmic work.
-KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5}
+# When both run as one launch (fa_bwd_grad_kernel) it does all five products
+# (2.5x forward) and executes seven (3.5x).
+KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5,
+                       "fa_bwd_grad_kernel": 2.5}
 # tile products each kernel executes, as multiples of the forward (2 products)
-KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5}
+KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5,
+                        "fa_bwd_grad_kernel": 3.5}
 
 
 def max_over_ranks(x, world, device=None):

@@ -23,6 +23,7 @@ __all__ = [
     "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
     "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_noalloc",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "fa_profile_enable", "fa_profile_read",
@@ -62,6 +63,10 @@ def lib() -> ctypes.CDLL:
             vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
             L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp]
             L.fa_fwd.restype = i
+            L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
+            L.fa_fwd_splitkv_workspace_bytes.restype = sz
+            L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
+            L.fa_fwd_splitkv.restype = i
             L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
             L.fa_bwd_workspace_bytes.restype = sz
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
@@ -132,6 +137,25 @@ def fa_fwd(q, k, v, o, lse, causal=False, scale=None, key_bias=None, stream=None
                       int(bool(causal)), float(scale), _dtype_code(q), _ptr(key_bias),
                       _stream_ptr(stream))
     _check(st, "fa_fwd")
+
+
+def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits) -> int:
+    return int(lib().fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, num_splits, workspace, causal=False, scale=None,
+                   key_bias=None, stream=None):
+    """Split-KV forward (few queries, many keys) into caller-owned o, lse,
+    with a caller-owned workspace of fa_fwd_splitkv_workspace_bytes() bytes."""
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
+                              int(bool(causal)), float(scale), _dtype_code(q), _ptr(key_bias),
+                              int(num_splits), _ptr(workspace), nbytes, _stream_ptr(stream))
+    _check(st, "fa_fwd_splitkv")
 
 
 def fa_bwd_workspace_bytes(B, H, Nq, Nk, D) -> int:

@@ -217,6 +217,66 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int D, int num_splits) {
+    (void)Nk;
+    if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128) || num_splits < 1 || num_splits > 256) return 0;
+    const size_t rows = static_cast<size_t>(B) * H * Nq * num_splits;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return up(rows * D * sizeof(float)) + up(rows * sizeof(float)) + 256;
+}
+
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                   int Nq, int Nk, int D, int causal, float scale, int dtype, const float *key_bias,
+                   int num_splits, void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
+    if (Nq == 0) return FA_OK;
+    if (num_splits == 1 || Nk == 0)
+        return fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, causal, scale, dtype, key_bias, stream);
+    if (!q || !o || !lse || !k || !v) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (key_bias && !aligned16(key_bias)) || !aligned16(workspace))
+        return FA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits))
+        return FA_ERR_WORKSPACE;
+    const long long units = static_cast<long long>(B) * H * ((Nq + 255) / 256) * num_splits;
+    if (units > INT32_MAX) return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    const long long BH = static_cast<long long>(B) * H;
+    fa::FwdTensorMaps tm;
+    if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.o, o, bf16, D, Nq, BH, 32)) != FA_OK) return st;
+    const size_t rows = static_cast<size_t>(BH) * Nq * num_splits;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    fa::FwdParams p;
+    p.B = B;
+    p.H = H;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.n_mblocks = (Nq + 255) / 256;
+    p.causal_off = Nk - Nq;
+    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    p.bias = key_bias;
+    p.lse = lse;
+    p.err = err;
+    p.timeout_ns = kDefaultTimeoutNs;
+    const int tiles = (Nk + 127) / 128;
+    p.num_splits = num_splits;
+    p.tiles_per_split = (tiles + num_splits - 1) / num_splits;
+    p.o_part = static_cast<float *>(workspace);
+    p.lse_part = reinterpret_cast<float *>(static_cast<char *>(workspace) + up(rows * D * sizeof(float)));
+    cudaError_t e = fa::launch_fwd_split(tm, p, D, bf16, causal != 0, key_bias != nullptr, o, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
     (void)Nk;
     if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128)) return 0;

@@ -12,16 +12,18 @@
 //   dS = P * (dP - D)  with D_i = sum_j P_ij dP_ij = rowsum(dO * O)
 //   dQ = scale dS K    dK = scale dS^T Q
 //
-// Three kernels on one stream, none of which stores S, P or dS:
+// Three steps on one stream, none of which stores S, P or dS:
 //   1. fa_bwd_pre_kernel   D_i = rowsum(dO * O) (fp32, the caller's workspace).
-//   2. fa_bwd_dkdv_kernel  one CTA per (b, h, 128-key tile); for every query
+// Kernels 2 and 3 run as the two kinds of block of one launch
+// (fa_bwd_grad_kernel), interleaved heaviest first.
+//   2. dK/dV blocks        one CTA per (b, h, 128-key tile); for every query
 //      tile j that can see these keys:
 //        S^T  = K Q_j^T, dP^T = V dO_j^T           tcgen05.mma -> tensor memory
 //        P^T  = 2^(S^T qk_scale + bias - LSE_2)     one thread per key row
 //        dS^T = P^T * (dP^T - D_j)
 //        dV  += P^T dO_j,  dK += dS^T Q_j           A operands from tensor memory
 //      dK (x scale) and dV are written once at the end.
-//   3. fa_bwd_dq_kernel    one CTA per (b, h, 128-query tile); for every key
+//   3. dQ blocks           one CTA per (b, h, 128-query tile); for every key
 //      tile j it can see: S = Q K_j^T, dP = dO V_j^T, P and dS as above (one
 //      thread per query row), dQ += dS K_j; dQ (x scale) written once.
 // dQ is therefore computed without atomics and is bitwise deterministic; the
@@ -220,20 +222,11 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 // they go straight on to phase 1 of j+1.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-__global__ void __launch_bounds__(kThreads, 1)
-fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                   const BwdParams p) {
+__device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                         const CUtensorMap &tm_v, const CUtensorMap &tm_do,
+                                         const CUtensorMap &tm_dk, const CUtensorMap &tm_dv,
+                                         const BwdParams &p, uint8_t *smem, int unit) {
     using L = DkdvLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment is needed by the 128-byte swizzle atoms; the dynamic
-    // shared window starts aligned when the kernel has no static shared memory.
-    if ((smem_u32(smem_raw) & 1023u) != 0) {
-        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
-        return;
-    }
-    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -243,8 +236,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     // ---- work unit: the key tiles that see the most query tiles come first
     const int BH = p.B * p.H;
-    const int t = blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    const int t = unit / BH;
+    const int bh = unit % BH;
     const int kv0 = t * kBK;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
     int j_begin = 0;
@@ -577,17 +570,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 // overlap dQ(j) and dP(j+1).
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-__global__ void __launch_bounds__(kThreads, 1)
-fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+__device__ __forceinline__ void dq_cta(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                       const CUtensorMap &tm_v, const CUtensorMap &tm_do,
+                                       const CUtensorMap &tm_dq, const BwdParams &p, uint8_t *smem,
+                                       int unit) {
     using L = DqLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    if ((smem_u32(smem_raw) & 1023u) != 0) {
-        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
-        return;
-    }
-    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -598,8 +585,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ---- work unit: query tiles that see the most key tiles come first
     const int BH = p.B * p.H;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
-    const int qt = (n_q_all - 1) - blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    const int qt = (n_q_all - 1) - unit / BH;
+    const int bh = unit % BH;
     const int q0 = qt * kBQ;
     const int n_kv_all = (p.Nk + kBK - 1) / kBK;
     int n = n_kv_all;
@@ -925,32 +912,60 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
+// ---------------------------------------------------------------------------
+// One launch for both gradient kernels.  They are independent (both only read
+// Q, K, V, dO, LSE and D), so a single grid whose blocks alternate between a
+// dK/dV unit and a dQ unit, each list heaviest first, lets the block scheduler
+// balance the two together (longest units first overall).
+// ---------------------------------------------------------------------------
+__host__ __device__ inline void grad_unit(int idx, int n_dkdv, int n_dq, int *kind, int *unit) {
+    const int both = 2 * (n_dkdv < n_dq ? n_dkdv : n_dq);
+    if (idx < both) {
+        *kind = idx & 1;
+        *unit = idx >> 1;
+    } else {
+        const int rest = idx - both;
+        *kind = n_dkdv > n_dq ? 0 : 1;
+        *unit = both / 2 + rest;
+    }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p, int n_dkdv, int n_dq) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment is needed by the 128-byte swizzle atoms; the dynamic
+    // shared window starts aligned when the kernel has no static shared memory.
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
+        return;
+    }
+    int kind, unit;
+    grad_unit(blockIdx.x, n_dkdv, n_dq, &kind, &unit);
+    if (kind == 0)
+        dkdv_cta<D, BF16, CAUSAL, HAS_BIAS>(tm_q, tm_k, tm_v, tm_do, tm_dk, tm_dv, p, smem_raw, unit);
+    else
+        dq_cta<D, BF16, CAUSAL, HAS_BIAS>(tm_q, tm_k, tm_v, tm_do, tm_dq, p, smem_raw, unit);
+}
+
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
-    {
-        using L = DkdvLayout<D>;
-        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-        if (e != cudaSuccess) return e;
-        const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
-        prof_begin(stream, "fa_bwd_dkdv_kernel");
-        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, p);
-        prof_end(stream);
-        note_launch();
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    {
-        using L = DqLayout<D>;
-        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-        if (e != cudaSuccess) return e;
-        const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
-        prof_begin(stream, "fa_bwd_dq_kernel");
-        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dq, p);
-        prof_end(stream);
-        note_launch();
-        return cudaGetLastError();
-    }
+    constexpr int kSmem = DkdvLayout<D>::kBytes > DqLayout<D>::kBytes ? DkdvLayout<D>::kBytes
+                                                                      : DqLayout<D>::kBytes;
+    auto kern = fa_bwd_grad_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    const int n_dkdv = ((p.Nk + kBK - 1) / kBK) * p.B * p.H;
+    const int n_dq = ((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
+    prof_begin(stream, "fa_bwd_grad_kernel");
+    kern<<<static_cast<unsigned>(n_dkdv + n_dq), kThreads, kSmem, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk,
+                                                                           tm.dv, tm.dq, p, n_dkdv, n_dq);
+    prof_end(stream);
+    note_launch();
+    return cudaGetLastError();
 }
 
 template <int D, bool BF16>

@@ -110,7 +110,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -128,18 +128,29 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int lane = threadIdx.x & 31;
 
     // ---- work unit: heaviest (last) query blocks first so that the hardware
-    // block scheduler hands the long causal units out early.
+    // block scheduler hands the long causal units out early.  With SPLIT, the
+    // unit also names one contiguous range of key tiles.
     const int BH = p.B * p.H;
-    const int unit = blockIdx.x;
+    int unit = blockIdx.x;
+    int split = 0;
+    if (SPLIT) {
+        split = unit % p.num_splits;
+        unit /= p.num_splits;
+    }
     const int mb = (p.n_mblocks - 1) - unit / BH;
     const int bh = unit % BH;
     const int m0 = mb * 2 * kBM;
     const int n_kv_all = (p.Nk + kBN - 1) / kBN;
-    int n_kv = n_kv_all;
+    int n_kv = n_kv_all;      // key tiles this block may see
     if (CAUSAL) {
         const int last_row = min(m0 + 2 * kBM - 1, p.Nq - 1);
         const int lim = last_row + p.causal_off;
         n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kBN + 1);
+    }
+    int kv_first = 0;         // first key tile of this unit
+    if (SPLIT) {
+        kv_first = split * p.tiles_per_split;
+        n_kv = max(0, min(n_kv, kv_first + p.tiles_per_split) - kv_first);
     }
 
     // ---- set-up
@@ -198,12 +209,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sbase + L::kK + s * L::kTileBytes + c * L::kChunkBytes, &tm_k,
-                                bar(L::kKFull + s), c * 64, j * kBN, bh);
+                                bar(L::kKFull + s), c * 64, (kv_first + j) * kBN, bh);
                 if (!mbar_wait(bar(L::kVEmpty + s), ph ^ 1, wctx)) { ok = false; issued = 2 * j + 1; break; }
                 mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTileBytes);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sbase + L::kV + s * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                bar(L::kVFull + s), c * 64, j * kBN, bh);
+                                bar(L::kVFull + s), c * 64, (kv_first + j) * kBN, bh);
                 issued = 2 * j + 2;
             }
             if (!ok) {
@@ -317,7 +328,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const int kv0 = j * kBN;
+            const int kv0 = (kv_first + j) * kBN;
             {
                 const bool got = mbar_wait(bar(L::kSFull + i), j & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -426,7 +437,30 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             ok = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
-        if (ok) {
+        if (ok && SPLIT) {
+            // partial result of this key range: O_s = o / l (fp32), LSE_s
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const size_t prow = (static_cast<size_t>(split) * BH + bh) * p.Nq + qrow;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t orr[32];
+                if (n_kv > 0) {
+                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                }
+                if (qrow < p.Nq) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + prow * D + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
+                                             __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
+                }
+            }
+            if (qrow < p.Nq)
+                p.lse_part[prow] = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : neg_inf();
+        } else if (ok) {
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             uint8_t *stage = smem + L::kQ + i * L::kTileBytes;   // Q_i is dead now
 #pragma unroll
@@ -477,6 +511,48 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
+// Merge of the split-KV partials, one warp per query row:
+//   LSE = m + ln sum_s exp(LSE_s - m),  O = sum_s exp(LSE_s - m) O_s / sum_s exp(LSE_s - m)
+// with m = max_s LSE_s (all -inf: the row saw no key, O = 0, LSE = -inf).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const float *__restrict__ o_part,
+                                                             const float *__restrict__ lse_part,
+                                                             uint16_t *__restrict__ o, float *__restrict__ lse,
+                                                             long long rows, int num_splits) {
+    constexpr int kPer = D / 32;   // values per lane (2 or 4)
+    const int lane = threadIdx.x & 31;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+        float m = neg_inf();
+        for (int s = 0; s < num_splits; ++s) m = fmaxf(m, lse_part[s * rows + r]);
+        float acc[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+        float wsum = 0.f;
+        if (m != neg_inf()) {
+            for (int s = 0; s < num_splits; ++s) {
+                const float ls = lse_part[s * rows + r];
+                if (ls == neg_inf()) continue;
+                const float w = __expf(ls - m);
+                wsum += w;
+                const float *src = o_part + (s * rows + r) * D + lane * kPer;
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        uint32_t packed[kPer / 2];
+#pragma unroll
+        for (int e = 0; e < kPer / 2; ++e) packed[e] = pack2<BF16>(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        uint16_t *dst = o + r * D + lane * kPer;
+        if constexpr (kPer == 4)
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+        else
+            *reinterpret_cast<uint32_t *>(dst) = packed[0];
+        if (lane == 0) lse[r] = wsum > 0.f ? m + __logf(wsum) : neg_inf();
+    }
+}
+
 // Rows with no key at all (Nk == 0): O = 0, LSE = -inf.
 template <typename T>
 __global__ void fa_fwd_empty_kernel(T *o, float *lse, size_t n_rows, int D) {
@@ -501,6 +577,35 @@ cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, cudaStream
     return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, void *o, cudaStream_t stream) {
+    using L = FwdLayout<D>;
+    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, HAS_BIAS, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H * p.num_splits;
+    prof_begin(stream, "fa_fwd_split_kernel");
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    prof_end(stream);
+    note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
+    const unsigned cgrid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+    prof_begin(stream, "fa_fwd_combine_kernel");
+    fa_fwd_combine_kernel<D, BF16><<<cgrid, 256, 0, stream>>>(p.o_part, p.lse_part, static_cast<uint16_t *>(o),
+                                                               p.lse, rows, p.num_splits);
+    prof_end(stream);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_split_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias, void *o,
+                           cudaStream_t s) {
+    if (causal) return bias ? launch_split_t<D, BF16, true, true>(tm, p, o, s) : launch_split_t<D, BF16, true, false>(tm, p, o, s);
+    return bias ? launch_split_t<D, BF16, false, true>(tm, p, o, s) : launch_split_t<D, BF16, false, false>(tm, p, o, s);
+}
+
 template <int D, bool BF16>
 cudaError_t launch_fwd_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias,
                          cudaStream_t s) {
@@ -516,6 +621,14 @@ cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool 
                              : launch_fwd_d<64, false>(tm, p, causal, has_bias, stream);
     return bf16 ? launch_fwd_d<128, true>(tm, p, causal, has_bias, stream)
                 : launch_fwd_d<128, false>(tm, p, causal, has_bias, stream);
+}
+
+cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                             bool has_bias, void *o, cudaStream_t stream) {
+    if (D == 64) return bf16 ? launch_split_d<64, true>(tm, p, causal, has_bias, o, stream)
+                             : launch_split_d<64, false>(tm, p, causal, has_bias, o, stream);
+    return bf16 ? launch_split_d<128, true>(tm, p, causal, has_bias, o, stream)
+                : launch_split_d<128, false>(tm, p, causal, has_bias, o, stream);
 }
 
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16, cudaStream_t stream) {

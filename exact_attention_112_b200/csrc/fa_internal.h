@@ -19,6 +19,11 @@ struct FwdParams {
     float *lse;                    // [B*H, Nq]
     int *err;                      // device error word
     unsigned long long timeout_ns; // limit of every device-side wait
+    // split-KV only: key tiles [s * tiles_per_split, (s + 1) * tiles_per_split)
+    int num_splits;
+    int tiles_per_split;
+    float *o_part;                 // [num_splits, B*H, Nq, D] fp32
+    float *lse_part;               // [num_splits, B*H, Nq]
 };
 
 struct FwdTensorMaps {
@@ -56,6 +61,8 @@ void prof_end(cudaStream_t stream);
 
 cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                        bool has_bias, cudaStream_t stream);
+cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                             bool has_bias, void *o, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,
                              cudaStream_t stream);
 

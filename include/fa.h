@@ -78,6 +78,26 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            int dtype, const float *key_bias, void *stream);
 
 /*
+ * Split-KV forward, for few query rows and many keys (decoding): the keys are
+ * cut into num_splits contiguous ranges of whole 128-key tiles, each range is
+ * processed by its own CTAs into a partial (O_s, LSE_s) in fp32, and a second
+ * kernel merges the partials with the associative log-sum-exp merge
+ *   LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s
+ * (the "secretly associative" softmax merge of the algebra digest,
+ * setupai.cc, "Mastering FlashAttention: The Algebraic Foundation").  Same
+ * arguments, layouts and results as fa_fwd() plus:
+ *   num_splits   1 .. 256 (1 is allowed and equals fa_fwd());
+ *   workspace    device memory of fa_fwd_splitkv_workspace_bytes() bytes,
+ *                16-byte aligned, caller-owned; contents on entry irrelevant.
+ * A split whose keys are all masked for a row contributes LSE_s = -inf.
+ */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int D, int num_splits);
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int H, int Nq, int Nk, int D, int causal, float scale,
+                   int dtype, const float *key_bias, int num_splits, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of device scratch fa_bwd() needs for these sizes: the per-row term
  * D_i = rowsum(dO * O), one float32 per query row (O(n) memory).
  */
