@@ -12,18 +12,16 @@
 //   dS = P * (dP - D)  with D_i = sum_j P_ij dP_ij = rowsum(dO * O)
 //   dQ = scale dS K    dK = scale dS^T Q
 //
-// Three steps on one stream, none of which stores S, P or dS:
+// Three kernels on one stream, none of which stores S, P or dS:
 //   1. fa_bwd_pre_kernel   D_i = rowsum(dO * O) (fp32, the caller's workspace).
-// Kernels 2 and 3 run as the two kinds of block of one launch
-// (fa_bwd_grad_kernel), interleaved heaviest first.
-//   2. dK/dV blocks        one CTA per (b, h, 128-key tile); for every query
+//   2. fa_bwd_dkdv_kernel  one CTA per (b, h, 128-key tile); for every query
 //      tile j that can see these keys:
 //        S^T  = K Q_j^T, dP^T = V dO_j^T           tcgen05.mma -> tensor memory
 //        P^T  = 2^(S^T qk_scale + bias - LSE_2)     one thread per key row
 //        dS^T = P^T * (dP^T - D_j)
 //        dV  += P^T dO_j,  dK += dS^T Q_j           A operands from tensor memory
 //      dK (x scale) and dV are written once at the end.
-//   3. dQ blocks           one CTA per (b, h, 128-query tile); for every key
+//   3. fa_bwd_dq_kernel    one CTA per (b, h, 128-query tile); for every key
 //      tile j it can see: S = Q K_j^T, dP = dO V_j^T, P and dS as above (one
 //      thread per query row), dQ += dS K_j; dQ (x scale) written once.
 // dQ is therefore computed without atomics and is bitwise deterministic; the
@@ -31,10 +29,9 @@
 // tiles instead of 5).
 //
 // Tensor memory of the dK/dV kernel (lane = key row):
-//   cols [0,128)      S^T (fp32)
-//   cols [128,256)    dP^T (fp32); then, in the 64 columns each recompute
-//                     warpgroup read, P^T (16-bit pairs) in the first 32 and
-//                     dS^T (16-bit pairs) in the next 32
+//   cols [0,128)      S^T (fp32); then P^T (16-bit pairs) in the first 32 of
+//                     the 64 columns each recompute warpgroup read
+//   cols [128,256)    dP^T (fp32); then dS^T (16-bit pairs) likewise
 //   cols [256,256+D)  dV accumulator,  cols [256+D,256+2D) dK accumulator
 // Tensor memory of the dQ kernel (lane = query row):
 //   cols [0,128), [128,256)  S of two consecutive key tiles (fp32); dS
@@ -96,11 +93,11 @@ struct DkdvLayout {
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr uint32_t kTmemCols = 512;
-    // Each recompute warpgroup g writes its 16-bit results only into the dP^T
-    // columns it has read itself, 128 + [64g, 64g+64): P^T pairs in the first
-    // 32 of them, dS^T pairs in the next 32.  The S^T columns are therefore
-    // free as soon as phase 1 has loaded them.
-    static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 128, kColDS = 160, kColDV = 256,
+    // Each recompute warpgroup g writes its 16-bit results only into columns
+    // it has read itself: P^T pairs over its S^T columns [64g, 64g+32) (phase
+    // 1), dS^T pairs over its dP^T columns 128 + [64g, 64g+32) (phase 2).  So
+    // S^T(j+1) only has to wait for dV(j), and dP^T(j+1) only for dK(j).
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 0, kColDS = 128, kColDV = 256,
                               kColDK = 256 + D;
 };
 
@@ -215,18 +212,27 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 // 2. dK, dV for one 128-key tile per CTA.
 //
 // MMA issue order per query tile j (one thread, in-order tensor pipe):
-//     S^T(j+1)           once phase 1 of j has loaded S^T(j) into registers
-//     dV(j), dK(j)       once phase 2 of j has put P^T, dS^T in tensor memory
+//     dV(j)        once phase 1 of j has put P^T over the S^T columns
+//     S^T(j+1)
+//     dK(j)        once phase 2 of j has put dS^T over the dP^T columns
 //     dP^T(j+1)
-// so S^T(j+1) is computed while the recompute warps run phase 2 of j, and
-// they go straight on to phase 1 of j+1.
+// so S^T(j+1) runs during phase 2 of j and dP^T(j+1) during phase 1 of j+1.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-__device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                         const CUtensorMap &tm_v, const CUtensorMap &tm_do,
-                                         const CUtensorMap &tm_dk, const CUtensorMap &tm_dv,
-                                         const BwdParams &p, uint8_t *smem, int unit) {
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                   const BwdParams p) {
     using L = DkdvLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment is needed by the 128-byte swizzle atoms; the dynamic
+    // shared window starts aligned when the kernel has no static shared memory.
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
+        return;
+    }
+    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -236,8 +242,8 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensor
 
     // ---- work unit: the key tiles that see the most query tiles come first
     const int BH = p.B * p.H;
-    const int t = unit / BH;
-    const int bh = unit % BH;
+    const int t = blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
     const int kv0 = t * kBK;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
     int j_begin = 0;
@@ -380,29 +386,30 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensor
                 const int s2 = (jj + 1) & 1;
                 const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
                 const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
-                // S^T(j+1) into the S^T columns, free once phase 1 of j has read them
+                // dV += P^T dO   (A: P^T over the S^T columns; B: dO rows, MN-major)
                 if (!mbar_wait(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
-                if (jj + 1 < nq) {
-                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_st(s2);
-                }
-                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
-                // dV += P^T dO   (A: P^T in tensor memory; B: dO rows, MN-major)
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
                     umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + (kk >> 2) * 64 + (kk & 3) * 8,
                                 smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
-                // dK += dS^T Q   (A: dS^T in tensor memory; B: Q rows, MN-major)
+                // S^T(j+1) over P^T(j) (read by dV(j) just before, in order)
+                if (jj + 1 < nq) {
+                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_st(s2);
+                }
+                // dK += dS^T Q   (A: dS^T over the dP^T columns; B: Q rows, MN-major)
+                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBQ / 16; ++kk)
                     umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + (kk >> 2) * 64 + (kk & 3) * 8,
                                 smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
                                 (jj > 0 || kk > 0) ? 1u : 0u);
                 if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
-                // dP^T(j+1) over the P^T / dS^T of j (read by dV(j), dK(j) just before)
+                // dP^T(j+1) over dS^T(j) (read by dK(j) just before, in order)
                 if (jj + 1 < nq) issue_dpt(s2);
             }
             umma_commit(bar(L::kAccFull));
@@ -433,7 +440,8 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensor
             const int s = jj & 1;
             const int qg = (j_begin + jj) * kBQ + 64 * g;     // first query of this thread's half
             const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256 + 64 * g;
-            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2), kept in registers
+            // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2): registers (fp32) and
+            // tensor memory (16-bit, the dV operand)
             {
                 const bool got = mbar_wait(bar(L::kSFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -467,43 +475,41 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensor
                     pr[4 * e4 + 2] = ex2_approx(x23.x);
                     pr[4 * e4 + 3] = ex2_approx(x23.y);
                 }
+                // P^T (16-bit) over the first 32 of this thread's S^T columns
+                uint32_t pp[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pp[e] = pack2<BF16>(pr[2 * e], pr[2 * e + 1]);
+                tmem_st32dp_x32(tl + L::kColP + 64 * g, pp);
             }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(L::kPTFull));   // S^T loaded: its columns may be overwritten
-            // ---- phase 2: dS^T = P^T (dP^T - D); P^T and dS^T (16-bit) -> the
-            // dP^T columns this thread has just read
+            mbar_arrive(bar(L::kPTFull));
+            // ---- phase 2: dS^T = P^T (dP^T - D), 16-bit, over the dP^T columns
+            // this thread has just read
             {
                 const bool got = mbar_wait(bar(L::kDPFull), jj & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
             {
-                // two halves of 32 columns keep the live registers low; every
-                // dP^T column of this thread is loaded before anything is stored
                 uint32_t dpv[64];
                 tmem_ld32dp_x64_wait(tl + L::kColDP + 64 * g, dpv);
                 const float4 *d4 = reinterpret_cast<const float4 *>(rowbuf + 128);
+                uint32_t dd[32];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pp[16], dd[16];
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 dv = d4[8 * h + e4];
-                        const int e = 32 * h + 4 * e4;
-                        pp[2 * e4] = pack2<BF16>(pr[e], pr[e + 1]);
-                        pp[2 * e4 + 1] = pack2<BF16>(pr[e + 2], pr[e + 3]);
-                        const float2 d01 = __fmul2_rn(make_float2(pr[e], pr[e + 1]),
-                                                      __fadd2_rn(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
-                                                                 make_float2(-dv.x, -dv.y)));
-                        const float2 d23 = __fmul2_rn(make_float2(pr[e + 2], pr[e + 3]),
-                                                      __fadd2_rn(make_float2(__uint_as_float(dpv[e + 2]), __uint_as_float(dpv[e + 3])),
-                                                                 make_float2(-dv.z, -dv.w)));
-                        dd[2 * e4] = pack2<BF16>(d01.x, d01.y);
-                        dd[2 * e4 + 1] = pack2<BF16>(d23.x, d23.y);
-                    }
-                    tmem_st32dp_x16(tl + L::kColP + 64 * g + 16 * h, pp);
-                    tmem_st32dp_x16(tl + L::kColDS + 64 * g + 16 * h, dd);
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 dv = d4[e4];
+                    const int e = 4 * e4;
+                    const float2 d01 = __fmul2_rn(make_float2(pr[e], pr[e + 1]),
+                                                  __fadd2_rn(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                                             make_float2(-dv.x, -dv.y)));
+                    const float2 d23 = __fmul2_rn(make_float2(pr[e + 2], pr[e + 3]),
+                                                  __fadd2_rn(make_float2(__uint_as_float(dpv[e + 2]), __uint_as_float(dpv[e + 3])),
+                                                             make_float2(-dv.z, -dv.w)));
+                    dd[2 * e4] = pack2<BF16>(d01.x, d01.y);
+                    dd[2 * e4 + 1] = pack2<BF16>(d23.x, d23.y);
                 }
+                tmem_st32dp_x32(tl + L::kColDS + 64 * g, dd);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -570,11 +576,17 @@ __device__ __forceinline__ void dkdv_cta(const CUtensorMap &tm_q, const CUtensor
 // overlap dQ(j) and dP(j+1).
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-__device__ __forceinline__ void dq_cta(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                       const CUtensorMap &tm_v, const CUtensorMap &tm_do,
-                                       const CUtensorMap &tm_dq, const BwdParams &p, uint8_t *smem,
-                                       int unit) {
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using L = DqLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
+        return;
+    }
+    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -585,8 +597,8 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap &tm_q, const CUtensorMa
     // ---- work unit: query tiles that see the most key tiles come first
     const int BH = p.B * p.H;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
-    const int qt = (n_q_all - 1) - unit / BH;
-    const int bh = unit % BH;
+    const int qt = (n_q_all - 1) - blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
     const int q0 = qt * kBQ;
     const int n_kv_all = (p.Nk + kBK - 1) / kBK;
     int n = n_kv_all;
@@ -912,60 +924,32 @@ __device__ __forceinline__ void dq_cta(const CUtensorMap &tm_q, const CUtensorMa
     }
 }
 
-// ---------------------------------------------------------------------------
-// One launch for both gradient kernels.  They are independent (both only read
-// Q, K, V, dO, LSE and D), so a single grid whose blocks alternate between a
-// dK/dV unit and a dQ unit, each list heaviest first, lets the block scheduler
-// balance the two together (longest units first overall).
-// ---------------------------------------------------------------------------
-__host__ __device__ inline void grad_unit(int idx, int n_dkdv, int n_dq, int *kind, int *unit) {
-    const int both = 2 * (n_dkdv < n_dq ? n_dkdv : n_dq);
-    if (idx < both) {
-        *kind = idx & 1;
-        *unit = idx >> 1;
-    } else {
-        const int rest = idx - both;
-        *kind = n_dkdv > n_dq ? 0 : 1;
-        *unit = both / 2 + rest;
-    }
-}
-
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-__global__ void __launch_bounds__(kThreads, 1)
-fa_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p, int n_dkdv, int n_dq) {
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment is needed by the 128-byte swizzle atoms; the dynamic
-    // shared window starts aligned when the kernel has no static shared memory.
-    if ((smem_u32(smem_raw) & 1023u) != 0) {
-        if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrInternal);
-        return;
-    }
-    int kind, unit;
-    grad_unit(blockIdx.x, n_dkdv, n_dq, &kind, &unit);
-    if (kind == 0)
-        dkdv_cta<D, BF16, CAUSAL, HAS_BIAS>(tm_q, tm_k, tm_v, tm_do, tm_dk, tm_dv, p, smem_raw, unit);
-    else
-        dq_cta<D, BF16, CAUSAL, HAS_BIAS>(tm_q, tm_k, tm_v, tm_do, tm_dq, p, smem_raw, unit);
-}
-
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
-    constexpr int kSmem = DkdvLayout<D>::kBytes > DqLayout<D>::kBytes ? DkdvLayout<D>::kBytes
-                                                                      : DqLayout<D>::kBytes;
-    auto kern = fa_bwd_grad_kernel<D, BF16, CAUSAL, HAS_BIAS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    const int n_dkdv = ((p.Nk + kBK - 1) / kBK) * p.B * p.H;
-    const int n_dq = ((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
-    prof_begin(stream, "fa_bwd_grad_kernel");
-    kern<<<static_cast<unsigned>(n_dkdv + n_dq), kThreads, kSmem, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk,
-                                                                           tm.dv, tm.dq, p, n_dkdv, n_dq);
-    prof_end(stream);
-    note_launch();
-    return cudaGetLastError();
+    {
+        using L = DkdvLayout<D>;
+        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
+        prof_begin(stream, "fa_bwd_dkdv_kernel");
+        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dk, tm.dv, p);
+        prof_end(stream);
+        note_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        using L = DqLayout<D>;
+        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
+        prof_begin(stream, "fa_bwd_dq_kernel");
+        kern<<<grid, kThreads, L::kBytes, stream>>>(tm.q, tm.k, tm.v, tm.dO, tm.dq, p);
+        prof_end(stream);
+        note_launch();
+        return cudaGetLastError();
+    }
 }
 
 template <int D, bool BF16>
