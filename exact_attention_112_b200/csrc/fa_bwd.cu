@@ -21,9 +21,11 @@
 //        dS^T = P^T * (dP^T - D_j)
 //        dV  += P^T dO_j,  dK += dS^T Q_j           A operands from tensor memory
 //      dK (x scale) and dV are written once at the end.
-//   3. fa_bwd_dq_kernel    one CTA per (b, h, 128-query tile); for every key
-//      tile j it can see: S = Q K_j^T, dP = dO V_j^T, P and dS as above (one
-//      thread per query row), dQ += dS K_j; dQ (x scale) written once.
+//   3. fa_bwd_dq_kernel    one CTA per (b, h, 128-query tile); Q and dO are
+//      copied once into tensor memory; for every key tile j it can see:
+//      S = Q K_j^T, dP = dO V_j^T (A operands from tensor memory), P and dS as
+//      above (one thread per query row), dQ += dS K_j; dQ (x scale) written
+//      once.
 // dQ is therefore computed without atomics and is bitwise deterministic; the
 // price is recomputing S and dP in kernel 3 (7 tile products per pair of
 // tiles instead of 5).
@@ -34,10 +36,12 @@
 //   cols [128,256)    dP^T (fp32); then dS^T (16-bit pairs) likewise
 //   cols [256,256+D)  dV accumulator,  cols [256+D,256+2D) dK accumulator
 // Tensor memory of the dQ kernel (lane = query row):
-//   cols [0,128), [128,256)  S of two consecutive key tiles (fp32); dS
-//                            (16-bit pairs) overwrites the first 32 of each
-//                            warpgroup's 64 columns
-//   cols [256,384)    dP (fp32),   cols [384,384+D) dQ accumulator
+//   cols [0,128)      S (fp32)
+//   cols [128,256)    dP (fp32); then dS (16-bit pairs) in the first 32 of
+//                     the 64 columns each recompute warpgroup read
+//   cols [256,256+D)  dQ accumulator
+//   then Q and dO of the CTA's query tile as 16-bit pairs (D/2 columns each),
+//   the A operands of S and dP
 // Warp roles (12 warps): 0-7 recompute/gradient (one thread per tile row and
 // half of the tile's columns: warpgroup g owns columns [64g, 64g+64)), 8 TMA
 // producer, 9 MMA issuer, 10-11 idle (they complete the third warpgroup for
@@ -107,9 +111,9 @@ struct DqLayout {
     static constexpr int kChunkBytes = 128 * 128;
     static constexpr int kKStages = 3;
     static constexpr int kVStages = 2;
-    static constexpr int kQ = 0;
+    static constexpr int kQ = 0;                                 // Q, later the dQ staging
     static constexpr int kDO = kQ + kTileBytes;
-    static constexpr int kK = kDO + kTileBytes;                 // kKStages
+    static constexpr int kK = kDO + kTileBytes;                  // kKStages
     static constexpr int kV = kK + kKStages * kTileBytes;        // kVStages
     static constexpr int kBias = kV + kVStages * kTileBytes;     // kKStages x 128 f32
     static constexpr int kBar = kBias + kKStages * 128 * 4;
@@ -118,16 +122,21 @@ struct DqLayout {
     static constexpr int kKEmpty = 4;    // +stage (3)
     static constexpr int kVFull = 7;     // +stage (2)
     static constexpr int kVEmpty = 9;    // +stage (2)
-    static constexpr int kSFull = 11;    // +buffer (2)
+    static constexpr int kSFull = 11;
+    static constexpr int kSRead = 12;    // every recompute thread has loaded S(j)
     static constexpr int kDPFull = 13;
     static constexpr int kDSFull = 14;
-    static constexpr int kOFull = 15;
-    static constexpr int kDrain = 16;
-    static constexpr int kNumBars = 17;
+    static constexpr int kQDReady = 15;  // Q and dO are in tensor memory
+    static constexpr int kOFull = 16;
+    static constexpr int kDrain = 17;
+    static constexpr int kNumBars = 18;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColDP = 256, kColDQ = 384;
+    // S, dP (dS over its first 32 columns of each warpgroup half), dQ
+    // accumulator, then Q and dO as 16-bit pairs (the A operands of S and dP)
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColQ = 256 + D,
+                              kColDO = 256 + D + D / 2;
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -568,12 +577,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 // ---------------------------------------------------------------------------
 // 3. dQ for one 128-query tile per CTA.
 //
-// MMA issue order per key tile j:
-//     dQ(j)      once dS(j) is in tensor memory (S buffer j % 2)
-//     dP(j+1)    (the dP columns were read by the recompute of j)
-//     S(j+2)     into S buffer j % 2
-// so the exponentials of tile j+1 (whose S was computed one step earlier)
-// overlap dQ(j) and dP(j+1).
+// Q and dO are the same for every key tile of the CTA, so the recompute
+// warps copy them once into tensor memory and S = Q K_j^T and dP = dO V_j^T
+// read their A operand from there: per key tile only K_j and V_j are read
+// from shared memory.  MMA issue order per key tile j:
+//     S(j+1)     once the recompute warps have loaded S(j) into registers
+//     dQ(j)      once dS(j) is over the dP columns
+//     dP(j+1)    (over dS(j), read by dQ(j) just before, in order)
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -623,10 +633,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(bar(L::kVFull + s), 1);
             mbar_init(bar(L::kVEmpty + s), 1);
         }
-        mbar_init(bar(L::kSFull + 0), 1);
-        mbar_init(bar(L::kSFull + 1), 1);
+        mbar_init(bar(L::kSFull), 1);
+        mbar_init(bar(L::kSRead), kRecompute);
         mbar_init(bar(L::kDPFull), 1);
         mbar_init(bar(L::kDSFull), kRecompute);
+        mbar_init(bar(L::kQDReady), kRecompute);
         mbar_init(bar(L::kOFull), 1);
         mbar_init(bar(L::kDrain), 1);
         fence_mbar_init();
@@ -657,8 +668,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tma_load_3d(sbase + L::kDO + c * L::kChunkBytes, &tm_do, bar(L::kQFull), c * 64, q0, bh);
             }
         }
-        // K runs up to two tiles ahead of V (K_j is needed by S(j) one step
-        // before V_j is needed by dP(j)).
+        // K runs one tile ahead of V (K_j is needed by S(j), before dP(j)).
         for (int j = 0; j < n && ok; ++j) {
             const int ks = j % L::kKStages;
             const uint32_t kph = (j / L::kKStages) & 1;
@@ -731,29 +741,27 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0 && n > 0) {
             constexpr uint32_t idesc_s = idesc_f16_f32acc(BF16, kBQ, kBK, false, false);   // S, dP
             constexpr uint32_t idesc_dq = idesc_f16_f32acc(BF16, kBQ, D, false, true);     // dQ
-            const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO;
-            auto issue_s = [&](int j) {        // S_j = Q K_j^T into buffer j % 2
+            auto issue_s = [&](int j) {        // S_j = Q K_j^T   (A: Q in tensor memory)
                 const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
-                const uint32_t d = tmem + ((j & 1) ? L::kColS1 : L::kColS0);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024),
+                    umma_f16_ts(tmem + L::kColS, tmem + L::kColQ + kk * 8, smem_desc_sw128(sK + off, 16, 1024),
                                 idesc_s, kk > 0);
                 }
-                umma_commit(bar(L::kSFull + (j & 1)));
+                umma_commit(bar(L::kSFull));
             };
-            auto issue_dp = [&](int j) {       // dP_j = dO V_j^T
+            auto issue_dp = [&](int j) {       // dP_j = dO V_j^T   (A: dO in tensor memory)
                 const uint32_t sV = sbase + L::kV + (j % L::kVStages) * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(tmem + L::kColDP, smem_desc_sw128(sDO + off, 16, 1024),
-                                smem_desc_sw128(sV + off, 16, 1024), idesc_s, kk > 0);
+                    umma_f16_ts(tmem + L::kColDP, tmem + L::kColDO + kk * 8, smem_desc_sw128(sV + off, 16, 1024),
+                                idesc_s, kk > 0);
                 }
                 umma_commit(bar(L::kDPFull));
             };
-            bool ok = mbar_wait(bar(L::kQFull), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
+            bool ok = mbar_wait(bar(L::kQDReady), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
             if (ok) {
                 tc_fence_after();
                 issue_s(0);
@@ -763,38 +771,33 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 issue_dp(0);
                 if (2 < n) umma_commit(bar(L::kVEmpty + 0));
-                if (n > 1) {
-                    ok = mbar_wait(bar(L::kKFull + 1), 0, wctx);
-                    if (ok) {
-                        tc_fence_after();
-                        issue_s(1);
-                    }
-                }
             }
             for (int j = 0; j < n && ok; ++j) {
-                // dQ += dS_j K_j  (A: dS in tensor memory; B: K rows, MN-major)
+                // S(j+1) as soon as every recompute thread holds S(j) in registers
+                if (j + 1 < n) {
+                    const int js = j + 1;
+                    if (!mbar_wait(bar(L::kSRead), j & 1, wctx)) { ok = false; break; }
+                    if (!mbar_wait(bar(L::kKFull + js % L::kKStages), (js / L::kKStages) & 1, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_s(js);
+                }
+                // dQ += dS_j K_j  (A: dS over the dP columns; B: K rows, MN-major)
                 if (!mbar_wait(bar(L::kDSFull), j & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
-                const uint32_t a = tmem + ((j & 1) ? L::kColS1 : L::kColS0);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDQ, a + (kk >> 2) * 64 + (kk & 3) * 8,
-                                smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024),
-                                idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(tmem + L::kColDQ, tmem + L::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                                smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024), idesc_dq,
+                                (j > 0 || kk > 0) ? 1u : 0u);
                 if (j + 3 < n) umma_commit(bar(L::kKEmpty + j % L::kKStages));
+                // dP(j+1) over dS(j)
                 if (j + 1 < n) {
                     const int jv = j + 1;
                     if (!mbar_wait(bar(L::kVFull + jv % L::kVStages), (jv / L::kVStages) & 1, wctx)) { ok = false; break; }
                     tc_fence_after();
                     issue_dp(jv);
                     if (jv + 2 < n) umma_commit(bar(L::kVEmpty + jv % L::kVStages));
-                }
-                if (j + 2 < n) {
-                    const int js = j + 2;
-                    if (!mbar_wait(bar(L::kKFull + js % L::kKStages), (js / L::kKStages) & 1, wctx)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_s(js);
                 }
             }
             umma_commit(bar(L::kOFull));
@@ -817,6 +820,35 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int q = q0 + row;
         const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const float qk = p.qk_scale_log2;
+        bool ok = true;
+        if (n > 0) {
+            // Q (warpgroup 0) or dO (warpgroup 1) row of this thread: shared
+            // memory (128-byte swizzled tile) -> tensor memory, the A operand
+            // of S or dP for every key tile of the CTA
+            const bool got = mbar_wait(bar(L::kQFull), 0, wctx);
+            ok = __all_sync(0xffffffffu, got);
+            if (ok) {
+                const uint8_t *src = smem + (g ? L::kDO : L::kQ) + row * 128;
+                uint32_t rv[D / 2];
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                    for (int k16 = 0; k16 < 8; ++k16) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(src + c * L::kChunkBytes + ((k16 ^ (row & 7)) * 16));
+                        rv[c * 32 + 4 * k16 + 0] = u.x;
+                        rv[c * 32 + 4 * k16 + 1] = u.y;
+                        rv[c * 32 + 4 * k16 + 2] = u.z;
+                        rv[c * 32 + 4 * k16 + 3] = u.w;
+                    }
+                if constexpr (D == 128)
+                    tmem_st32dp_x64(tl + (g ? L::kColDO : L::kColQ), rv);
+                else
+                    tmem_st32dp_x32(tl + (g ? L::kColDO : L::kColQ), rv);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::kQDReady));
+        }
         float lse2 = pos_inf(), di = 0.f;
         if (q < p.Nq) {
             const float l = __ldg(p.lse + static_cast<size_t>(bh) * p.Nq + q);
@@ -825,12 +857,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // last key this row may see
         const int lim = CAUSAL ? min(q + p.causal_off, p.Nk - 1) : p.Nk - 1;
-        bool ok = true;
-        for (int j = 0; j < n; ++j) {
+        for (int j = 0; j < n && ok; ++j) {
             const int kg = j * kBK + 64 * g;                  // first key of this thread's half
-            const uint32_t tS = tl + ((j & 1) ? L::kColS1 : L::kColS0);
             {
-                const bool got = mbar_wait(bar(L::kSFull + (j & 1)), (j >> 1) & 1, wctx);
+                const bool got = mbar_wait(bar(L::kSFull), j & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
@@ -838,7 +868,9 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float pr[64];
             {
                 uint32_t sv[64];
-                tmem_ld32dp_x64_wait(tS + 64 * g, sv);
+                tmem_ld32dp_x64_wait(tl + L::kColS + 64 * g, sv);
+                tc_fence_before();
+                mbar_arrive(bar(L::kSRead));   // the S columns may now be overwritten
                 const float *bs = reinterpret_cast<const float *>(smem + L::kBias) +
                                   (j % L::kKStages) * 128 + 64 * g;
                 const bool edge = kg + 63 > lim;
@@ -860,7 +892,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     pr[e + 1] = ex2_approx(x.y);
                 }
             }
-            // ---- dS = P (dP - D) -> tensor memory (16-bit), over the S columns
+            // ---- dS = P (dP - D), 16-bit, over the dP columns this thread read
             {
                 const bool got = mbar_wait(bar(L::kDPFull), j & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -877,13 +909,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                 __fadd2_rn(make_float2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), nd2));
                     dd[e] = pack2<BF16>(d.x, d.y);
                 }
-                tmem_st32dp_x32(tS + 64 * g, dd);
+                tmem_st32dp_x32(tl + L::kColDP + 64 * g, dd);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::kDSFull));
         }
-        // ---- epilogue (warpgroup 0): dQ = scale * acc, 16-bit, staged in the (idle) Q buffer
+        // ---- epilogue (warpgroup 0): dQ = scale * acc, 16-bit, staged in the Q buffer
         if (g != 0) ok = false;
         if (ok && n > 0) {
             const bool got = mbar_wait(bar(L::kOFull), 0, wctx);
