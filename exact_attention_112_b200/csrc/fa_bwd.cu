@@ -737,71 +737,82 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
-        // ===================== MMA issuer =====================
-        if (lane == 0 && n > 0) {
+        // ===================== MMA issuer (whole warp; one elected lane issues) =====================
+        if (n > 0) {
             constexpr uint32_t idesc_s = idesc_f16_f32acc(BF16, kBQ, kBK, false, false);   // S, dP
             constexpr uint32_t idesc_dq = idesc_f16_f32acc(BF16, kBQ, D, false, true);     // dQ
             auto issue_s = [&](int j) {        // S_j = Q K_j^T   (A: Q in tensor memory)
-                const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
+                const uint64_t dk = smem_desc_sw128(sbase + L::kK + (j % L::kKStages) * L::kTileBytes, 16, 1024);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ts(tmem + L::kColS, tmem + L::kColQ + kk * 8, smem_desc_sw128(sK + off, 16, 1024),
-                                idesc_s, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_f16_ts(tmem + L::kColS, tmem + L::kColQ + kk * 8,
+                                    dk + (((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
+                    umma_commit(bar(L::kSFull));
                 }
-                umma_commit(bar(L::kSFull));
+                __syncwarp();
             };
             auto issue_dp = [&](int j) {       // dP_j = dO V_j^T   (A: dO in tensor memory)
-                const uint32_t sV = sbase + L::kV + (j % L::kVStages) * L::kTileBytes;
+                const uint64_t dv = smem_desc_sw128(sbase + L::kV + (j % L::kVStages) * L::kTileBytes, 16, 1024);
+                const bool release = j + 2 < n;
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ts(tmem + L::kColDP, tmem + L::kColDO + kk * 8, smem_desc_sw128(sV + off, 16, 1024),
-                                idesc_s, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_f16_ts(tmem + L::kColDP, tmem + L::kColDO + kk * 8,
+                                    dv + (((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
+                    umma_commit(bar(L::kDPFull));
+                    if (release) umma_commit(bar(L::kVEmpty + j % L::kVStages));
                 }
-                umma_commit(bar(L::kDPFull));
+                __syncwarp();
             };
-            bool ok = mbar_wait(bar(L::kQDReady), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
+            bool ok = mbar_wait_warp(bar(L::kQDReady), 0, wctx) && mbar_wait_warp(bar(L::kKFull + 0), 0, wctx);
             if (ok) {
                 tc_fence_after();
                 issue_s(0);
-                ok = mbar_wait(bar(L::kVFull + 0), 0, wctx);
+                ok = mbar_wait_warp(bar(L::kVFull + 0), 0, wctx);
             }
             if (ok) {
                 tc_fence_after();
                 issue_dp(0);
-                if (2 < n) umma_commit(bar(L::kVEmpty + 0));
             }
             for (int j = 0; j < n && ok; ++j) {
                 // S(j+1) as soon as every recompute thread holds S(j) in registers
                 if (j + 1 < n) {
                     const int js = j + 1;
-                    if (!mbar_wait(bar(L::kSRead), j & 1, wctx)) { ok = false; break; }
-                    if (!mbar_wait(bar(L::kKFull + js % L::kKStages), (js / L::kKStages) & 1, wctx)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(L::kSRead), j & 1, wctx)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(L::kKFull + js % L::kKStages), (js / L::kKStages) & 1, wctx)) { ok = false; break; }
                     tc_fence_after();
                     issue_s(js);
                 }
                 // dQ += dS_j K_j  (A: dS over the dP columns; B: K rows, MN-major)
-                if (!mbar_wait(bar(L::kDSFull), j & 1, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kDSFull), j & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sK = sbase + L::kK + (j % L::kKStages) * L::kTileBytes;
+                {
+                    const uint64_t dk = smem_desc_sw128(sbase + L::kK + (j % L::kKStages) * L::kTileBytes,
+                                                        L::kChunkBytes, 1024);
+                    const bool release = j + 3 < n;
+                    if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDQ, tmem + L::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                                smem_desc_sw128(sK + kk * 2048, L::kChunkBytes, 1024), idesc_dq,
-                                (j > 0 || kk > 0) ? 1u : 0u);
-                if (j + 3 < n) umma_commit(bar(L::kKEmpty + j % L::kKStages));
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_f16_ts(tmem + L::kColDQ, tmem + L::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                                        dk + ((kk * 2048) >> 4), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                        if (release) umma_commit(bar(L::kKEmpty + j % L::kKStages));
+                    }
+                    __syncwarp();
+                }
                 // dP(j+1) over dS(j)
                 if (j + 1 < n) {
                     const int jv = j + 1;
-                    if (!mbar_wait(bar(L::kVFull + jv % L::kVStages), (jv / L::kVStages) & 1, wctx)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(L::kVFull + jv % L::kVStages), (jv / L::kVStages) & 1, wctx)) { ok = false; break; }
                     tc_fence_after();
                     issue_dp(jv);
-                    if (jv + 2 < n) umma_commit(bar(L::kVEmpty + jv % L::kVStages));
                 }
             }
-            umma_commit(bar(L::kOFull));
-            umma_commit(bar(L::kDrain));
+            if (elect_one()) {
+                umma_commit(bar(L::kOFull));
+                umma_commit(bar(L::kDrain));
+            }
+            __syncwarp();
             WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
             volatile int zero = 0;
             drain.abort_flag = &zero;

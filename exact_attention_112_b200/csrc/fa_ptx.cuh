@@ -90,6 +90,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     return mbar_wait_slow(bar, parity, w);
 }
 
+// mbar_wait by every lane of a warp, with one outcome for the whole warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx &w) {
+    const bool got = mbar_wait(bar, parity, w);
+    return __all_sync(0xffffffffu, got);
+}
+
 // ----------------------------------------------------------------------------
 // TMA (tensor copies between global and shared memory)
 // ----------------------------------------------------------------------------
@@ -208,6 +214,20 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
+// One lane of a fully active warp (the lowest), chosen by elect.sync.  The MMA
+// roles run their loops with the whole warp, so that loop counters, stage
+// indices and descriptors are warp-uniform, and only the elected lane issues
+// tcgen05 instructions (commits included: they track that lane's MMAs).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
