@@ -356,34 +356,39 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
-        // ===================== MMA issuer =====================
-        if (lane == 0) {
+        // ===================== MMA issuer (whole warp; one elected lane issues) =====================
+        {
             constexpr uint32_t idesc_st = idesc_f16_f32acc(BF16, kBK, kBQ, false, false);  // S^T, dP^T
             constexpr uint32_t idesc_acc = idesc_f16_f32acc(BF16, kBK, D, false, true);    // dV, dK
-            const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
+            const uint64_t dK0 = smem_desc_sw128(sbase + L::kK, 16, 1024);
+            const uint64_t dV0 = smem_desc_sw128(sbase + L::kV, 16, 1024);
             auto issue_st = [&](int s) {    // S^T = K Q^T (both K-major)
-                const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
+                const uint64_t dq = smem_desc_sw128(sbase + L::kQ + s * L::kTileBytes, 16, 1024);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(tmem + L::kColS, smem_desc_sw128(sK + off, 16, 1024),
-                                smem_desc_sw128(sQ + off, 16, 1024), idesc_st, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+                        umma_f16_ss(tmem + L::kColS, dK0 + off, dq + off, idesc_st, kk > 0);
+                    }
+                    umma_commit(bar(L::kSFull));
                 }
-                umma_commit(bar(L::kSFull));
+                __syncwarp();
             };
             auto issue_dpt = [&](int s) {   // dP^T = V dO^T (both K-major)
-                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
+                const uint64_t ddo = smem_desc_sw128(sbase + L::kDO + s * L::kTileBytes, 16, 1024);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(tmem + L::kColDP, smem_desc_sw128(sV + off, 16, 1024),
-                                smem_desc_sw128(sDO + off, 16, 1024), idesc_st, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+                        umma_f16_ss(tmem + L::kColDP, dV0 + off, ddo + off, idesc_st, kk > 0);
+                    }
+                    umma_commit(bar(L::kDPFull));
                 }
-                umma_commit(bar(L::kDPFull));
+                __syncwarp();
             };
-            bool ok = mbar_wait(bar(L::kKVFull), 0, wctx);
+            bool ok = mbar_wait_warp(bar(L::kKVFull), 0, wctx);
             if (ok && nq > 0) {
-                ok = mbar_wait(bar(L::kQFull + 0), 0, wctx);
+                ok = mbar_wait_warp(bar(L::kQFull + 0), 0, wctx);
                 if (ok) {
                     tc_fence_after();
                     issue_st(0);
@@ -393,36 +398,48 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int jj = 0; jj < nq && ok; ++jj) {
                 const int s = jj & 1;
                 const int s2 = (jj + 1) & 1;
-                const uint32_t sQ = sbase + L::kQ + s * L::kTileBytes;
-                const uint32_t sDO = sbase + L::kDO + s * L::kTileBytes;
                 // dV += P^T dO   (A: P^T over the S^T columns; B: dO rows, MN-major)
-                if (!mbar_wait(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kPTFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
+                {
+                    const uint64_t ddo = smem_desc_sw128(sbase + L::kDO + s * L::kTileBytes, L::kChunkBytes, 1024);
+                    if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + (kk >> 2) * 64 + (kk & 3) * 8,
-                                smem_desc_sw128(sDO + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
-                                (jj > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBQ / 16; ++kk)
+                            umma_f16_ts(tmem + L::kColDV, tmem + L::kColP + (kk >> 2) * 64 + (kk & 3) * 8,
+                                        ddo + ((kk * 2048) >> 4), idesc_acc, (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    __syncwarp();
+                }
                 // S^T(j+1) over P^T(j) (read by dV(j) just before, in order)
                 if (jj + 1 < nq) {
-                    if (!mbar_wait(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(L::kQFull + s2), ((jj + 1) >> 1) & 1, wctx)) { ok = false; break; }
                     tc_fence_after();
                     issue_st(s2);
                 }
                 // dK += dS^T Q   (A: dS^T over the dP^T columns; B: Q rows, MN-major)
-                if (!mbar_wait(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kDSFull), jj & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
+                {
+                    const uint64_t dq = smem_desc_sw128(sbase + L::kQ + s * L::kTileBytes, L::kChunkBytes, 1024);
+                    const bool release = jj + 2 < nq;
+                    if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk)
-                    umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + (kk >> 2) * 64 + (kk & 3) * 8,
-                                smem_desc_sw128(sQ + kk * 2048, L::kChunkBytes, 1024), idesc_acc,
-                                (jj > 0 || kk > 0) ? 1u : 0u);
-                if (jj + 2 < nq) umma_commit(bar(L::kQEmpty + s));
+                        for (int kk = 0; kk < kBQ / 16; ++kk)
+                            umma_f16_ts(tmem + L::kColDK, tmem + L::kColDS + (kk >> 2) * 64 + (kk & 3) * 8,
+                                        dq + ((kk * 2048) >> 4), idesc_acc, (jj > 0 || kk > 0) ? 1u : 0u);
+                        if (release) umma_commit(bar(L::kQEmpty + s));
+                    }
+                    __syncwarp();
+                }
                 // dP^T(j+1) over dS^T(j) (read by dK(j) just before, in order)
                 if (jj + 1 < nq) issue_dpt(s2);
             }
-            umma_commit(bar(L::kAccFull));
-            umma_commit(bar(L::kDrain));
+            if (elect_one()) {
+                umma_commit(bar(L::kAccFull));
+                umma_commit(bar(L::kDrain));
+            }
+            __syncwarp();
             WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
             volatile int zero = 0;
             drain.abort_flag = &zero;

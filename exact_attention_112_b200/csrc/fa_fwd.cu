@@ -234,39 +234,45 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
-        // ===================== MMA issuer (one thread) =====================
-        if (lane == 0 && n_kv > 0) {
+        // ============ MMA issuer (whole warp; one elected lane issues) ============
+        if (n_kv > 0) {
             constexpr uint32_t idesc_qk = idesc_f16_f32acc(BF16, kBM, kBN, false, false);
             constexpr uint32_t idesc_pv = idesc_f16_f32acc(BF16, kBM, D, false, true);
-            auto issue_s = [&](int i, int stage) {
-                const uint32_t qa = sbase + L::kQ + i * L::kTileBytes;
-                const uint32_t ka = sbase + L::kK + stage * L::kTileBytes;
+            // S_i = Q_i K^T, then commit to `done` (and to `done2` if not 0)
+            auto issue_s = [&](int i, int stage, uint32_t done, uint32_t done2) {
+                const uint64_t dq = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
+                const uint64_t dk = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
                 const uint32_t d = tmem + (i ? L::kColS1 : L::kColS0);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(d, smem_desc_sw128(qa + off, 16, 1024),
-                                smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+                        umma_f16_ss(d, dq + off, dk + off, idesc_qk, kk > 0);
+                    }
+                    umma_commit(done);
+                    if (done2) umma_commit(done2);
                 }
+                __syncwarp();
             };
-            auto issue_pv = [&](int i, int stage, bool acc) {
-                const uint32_t va = sbase + L::kV + stage * L::kTileBytes;
+            // O_i += P_i V (A: P_i over the S_i columns), then commit to `done` if not 0
+            auto issue_pv = [&](int i, int stage, bool acc, uint32_t done) {
+                const uint64_t dv = smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
                 const uint32_t pa = tmem + (i ? L::kColS1 : L::kColS0);
                 const uint32_t d = tmem + (i ? L::kColO1 : L::kColO0);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    umma_f16_ts(d, pa + kk * 8, smem_desc_sw128(va + kk * 16 * 128, L::kChunkBytes, 1024),
-                                idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        umma_f16_ts(d, pa + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
+                                    (acc || kk > 0) ? 1u : 0u);
+                    if (done) umma_commit(done);
                 }
+                __syncwarp();
             };
-            bool ok = mbar_wait(bar(L::kQFull), 0, wctx) && mbar_wait(bar(L::kKFull + 0), 0, wctx);
+            bool ok = mbar_wait_warp(bar(L::kQFull), 0, wctx) && mbar_wait_warp(bar(L::kKFull + 0), 0, wctx);
             if (ok) {
                 tc_fence_after();
-                issue_s(0, 0);
-                umma_commit(bar(L::kSFull + 0));
-                issue_s(1, 0);
-                umma_commit(bar(L::kSFull + 1));
-                if (n_kv > 2) umma_commit(bar(L::kKEmpty + 0));
+                issue_s(0, 0, bar(L::kSFull + 0), 0u);
+                issue_s(1, 0, bar(L::kSFull + 1), n_kv > 2 ? bar(L::kKEmpty + 0) : 0u);
             }
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int s = j & 1;
@@ -274,32 +280,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const bool more = j + 1 < n_kv;
                 const int s2 = (j + 1) & 1;
                 const uint32_t ph2 = ((j + 1) >> 1) & 1;
-                if (!mbar_wait(bar(L::kVFull + s), ph, wctx)) { ok = false; break; }
-                if (!mbar_wait(bar(L::kPFull + 0), j & 1, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kVFull + s), ph, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kPFull + 0), j & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
-                issue_pv(0, s, j > 0);
+                issue_pv(0, s, j > 0, more ? 0u : bar(L::kOFull + 0));
                 if (more) {
-                    if (!mbar_wait(bar(L::kKFull + s2), ph2, wctx)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(L::kKFull + s2), ph2, wctx)) { ok = false; break; }
                     tc_fence_after();
-                    issue_s(0, s2);
-                    umma_commit(bar(L::kSFull + 0));
-                } else {
-                    umma_commit(bar(L::kOFull + 0));
+                    issue_s(0, s2, bar(L::kSFull + 0), 0u);
                 }
-                if (!mbar_wait(bar(L::kPFull + 1), j & 1, wctx)) { ok = false; break; }
+                if (!mbar_wait_warp(bar(L::kPFull + 1), j & 1, wctx)) { ok = false; break; }
                 tc_fence_after();
-                issue_pv(1, s, j > 0);
-                if (j + 2 < n_kv) umma_commit(bar(L::kVEmpty + s));
-                if (more) {
-                    issue_s(1, s2);
-                    umma_commit(bar(L::kSFull + 1));
-                    if (j + 3 < n_kv) umma_commit(bar(L::kKEmpty + s2));
-                } else {
+                issue_pv(1, s, j > 0, j + 2 < n_kv ? bar(L::kVEmpty + s) : 0u);
+                if (more)
+                    issue_s(1, s2, bar(L::kSFull + 1), j + 3 < n_kv ? bar(L::kKEmpty + s2) : 0u);
+                else if (elect_one())
                     umma_commit(bar(L::kOFull + 1));
-                }
+                __syncwarp();
             }
             // Every issued MMA must finish before tensor memory is released.
-            umma_commit(bar(L::kDrain));
+            if (elect_one()) umma_commit(bar(L::kDrain));
+            __syncwarp();
             WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
             volatile int zero = 0;
             drain.abort_flag = &zero;
