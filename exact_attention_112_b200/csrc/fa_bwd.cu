@@ -55,6 +55,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
@@ -73,6 +74,7 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kRegsRecompute = 192;
 constexpr uint32_t kRegsOther = 120;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kEmuEvery = 4;      // one pair of exponentials in kEmuEvery on the FMA pipe
 
 template <int D>
 struct DkdvLayout {
@@ -138,6 +140,10 @@ struct DqLayout {
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColQ = 256 + D,
                               kColDO = 256 + D + D / 2;
 };
+// The dynamic shared memory of a CTA is at most 227 KB; the kernels check at
+// run time that the window starts 1024-byte aligned, so no slack is reserved.
+static_assert(DkdvLayout<128>::kBytes <= 232448 && DkdvLayout<64>::kBytes <= 232448, "dK/dV shared memory");
+static_assert(DqLayout<128>::kBytes <= 232448 && DqLayout<64>::kBytes <= 232448, "dQ shared memory");
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
@@ -481,26 +487,41 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const float4 *l4 = reinterpret_cast<const float4 *>(rowbuf);
                 const float2 qk2 = make_float2(qk, qk);
                 const float2 b22 = make_float2(b2, b2);
+                // Without masked scores in this thread's columns, one pair in
+                // kEmuEvery takes the FMA-pipe exponential instead of MUFU.
+                auto make_p = [&](auto emu_tag) {
+                    constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-                for (int e4 = 0; e4 < 16; ++e4) {
-                    const float4 lv = l4[e4];
-                    // x = s qk + (bias - LSE_2), two columns per instruction
-                    const float2 c01 = __fadd2_rn(b22, make_float2(-lv.x, -lv.y));
-                    const float2 c23 = __fadd2_rn(b22, make_float2(-lv.z, -lv.w));
-                    float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4]), __uint_as_float(sv[4 * e4 + 1])), qk2, c01);
-                    float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])), qk2, c23);
-                    if (diag) {
-                        const int e = 4 * e4;
-                        if (key > qg + e + p.causal_off) x01.x = neg_inf();
-                        if (key > qg + e + 1 + p.causal_off) x01.y = neg_inf();
-                        if (key > qg + e + 2 + p.causal_off) x23.x = neg_inf();
-                        if (key > qg + e + 3 + p.causal_off) x23.y = neg_inf();
+                    for (int e4 = 0; e4 < 16; ++e4) {
+                        const float4 lv = l4[e4];
+                        // x = s qk + (bias - LSE_2), two columns per instruction
+                        const float2 c01 = __fadd2_rn(b22, make_float2(-lv.x, -lv.y));
+                        const float2 c23 = __fadd2_rn(b22, make_float2(-lv.z, -lv.w));
+                        float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4]), __uint_as_float(sv[4 * e4 + 1])), qk2, c01);
+                        float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])), qk2, c23);
+                        if (!kEmu && diag) {
+                            const int e = 4 * e4;
+                            if (key > qg + e + p.causal_off) x01.x = neg_inf();
+                            if (key > qg + e + 1 + p.causal_off) x01.y = neg_inf();
+                            if (key > qg + e + 2 + p.causal_off) x23.x = neg_inf();
+                            if (key > qg + e + 3 + p.causal_off) x23.y = neg_inf();
+                        }
+                        pr[4 * e4] = ex2_approx(x01.x);
+                        pr[4 * e4 + 1] = ex2_approx(x01.y);
+                        if (kEmu && (2 * e4 + 1) % kEmuEvery == kEmuEvery - 1) {
+                            const float2 p23 = exp2_fma2(x23);
+                            pr[4 * e4 + 2] = p23.x;
+                            pr[4 * e4 + 3] = p23.y;
+                        } else {
+                            pr[4 * e4 + 2] = ex2_approx(x23.x);
+                            pr[4 * e4 + 3] = ex2_approx(x23.y);
+                        }
                     }
-                    pr[4 * e4] = ex2_approx(x01.x);
-                    pr[4 * e4 + 1] = ex2_approx(x01.y);
-                    pr[4 * e4 + 2] = ex2_approx(x23.x);
-                    pr[4 * e4 + 3] = ex2_approx(x23.y);
-                }
+                };
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !diag && key < p.Nk))   // warp-uniform
+                    make_p(std::true_type{});
+                else
+                    make_p(std::false_type{});
                 // P^T (16-bit) over the first 32 of this thread's S^T columns
                 uint32_t pp[32];
 #pragma unroll
@@ -904,21 +925,36 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const bool edge = kg + 63 > lim;
                 const float2 qk2 = make_float2(qk, qk);
                 const float2 nl2 = make_float2(-lse2, -lse2);
+                // Without masked scores in this thread's columns, one pair in
+                // kEmuEvery takes the FMA-pipe exponential instead of MUFU.
+                auto make_p = [&](auto emu_tag) {
+                    constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float2 sc = make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
-                    float2 x;
-                    if constexpr (HAS_BIAS)
-                        x = __ffma2_rn(sc, qk2, __fadd2_rn(make_float2(bs[e], bs[e + 1]), nl2));
-                    else
-                        x = __ffma2_rn(sc, qk2, nl2);
-                    if (edge) {
-                        if (kg + e > lim) x.x = neg_inf();
-                        if (kg + e + 1 > lim) x.y = neg_inf();
+                    for (int e = 0; e < 64; e += 2) {
+                        const float2 sc = make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+                        float2 x;
+                        if constexpr (HAS_BIAS)
+                            x = __ffma2_rn(sc, qk2, __fadd2_rn(make_float2(bs[e], bs[e + 1]), nl2));
+                        else
+                            x = __ffma2_rn(sc, qk2, nl2);
+                        if (!kEmu && edge) {
+                            if (kg + e > lim) x.x = neg_inf();
+                            if (kg + e + 1 > lim) x.y = neg_inf();
+                        }
+                        if (kEmu && (e / 2) % kEmuEvery == kEmuEvery - 1) {
+                            const float2 pp = exp2_fma2(x);
+                            pr[e] = pp.x;
+                            pr[e + 1] = pp.y;
+                        } else {
+                            pr[e] = ex2_approx(x.x);
+                            pr[e + 1] = ex2_approx(x.y);
+                        }
                     }
-                    pr[e] = ex2_approx(x.x);
-                    pr[e + 1] = ex2_approx(x.y);
-                }
+                };
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !edge && q < p.Nq))   // warp-uniform
+                    make_p(std::true_type{});
+                else
+                    make_p(std::false_type{});
             }
             // ---- dS = P (dP - D), 16-bit, over the dP columns this thread read
             {

@@ -50,6 +50,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
@@ -69,6 +70,7 @@ constexpr uint32_t kRegsSoftmax = 192;
 constexpr uint32_t kRegsOther = 120;
 constexpr int kStages = 2;
 constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
+constexpr int kEmuEvery = 4;        // one pair of exponentials in kEmuEvery on the FMA pipe
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
@@ -393,24 +395,38 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
             // p = 2^(x - m), two columns per paired-fp32 instruction.  P goes
             // back into the S columns in two halves (every S value is already
-            // in registers), which keeps the live registers low.
+            // in registers), which keeps the live registers low.  On tiles
+            // without masked scores, one pair in kEmuEvery goes through the
+            // FMA-pipe exponential instead of MUFU.
             float2 lsum = make_float2(0.f, 0.f);
             const float2 neg_m2 = make_float2(-m_use, -m_use);
             const float2 qk2 = make_float2(qk, qk);
+            auto make_p = [&](auto emu_tag) {
+                constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
 #pragma unroll
-                for (int c2 = 0; c2 < 32; ++c2) {
-                    const int c = 64 * h + 2 * c2;
-                    const float2 xc = make_float2(x[c], x[c + 1]);
-                    const float2 a = HAS_BIAS ? __fadd2_rn(xc, neg_m2) : __ffma2_rn(xc, qk2, neg_m2);
-                    const float2 pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-                    lsum = __fadd2_rn(lsum, pp);
-                    pk[c2] = pack2<BF16>(pp.x, pp.y);
+                    for (int c2 = 0; c2 < 32; ++c2) {
+                        const int c = 64 * h + 2 * c2;
+                        const float2 xc = make_float2(x[c], x[c + 1]);
+                        const float2 a = HAS_BIAS ? __fadd2_rn(xc, neg_m2) : __ffma2_rn(xc, qk2, neg_m2);
+                        float2 pp;
+                        if (kEmu && c2 % kEmuEvery == kEmuEvery - 1)
+                            pp = exp2_fma2(a);
+                        else
+                            pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                        lsum = __fadd2_rn(lsum, pp);
+                        pk[c2] = pack2<BF16>(pp.x, pp.y);
+                    }
+                    tmem_st32dp_x32(tS + 32 * h, pk);
                 }
-                tmem_st32dp_x32(tS + 32 * h, pk);
-            }
+            };
+            // warp-uniform choice: make_p holds warp-collective tensor-memory stores
+            if (__all_sync(0xffffffffu, !HAS_BIAS && kv0 + kBN - 1 <= lim))
+                make_p(std::true_type{});
+            else
+                make_p(std::false_type{});
             const float l0 = lsum.x, l1 = lsum.y;
             l += l0 + l1;
             if (rescale && j > 0) {

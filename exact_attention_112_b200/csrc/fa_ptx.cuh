@@ -318,6 +318,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x for two values on the FMA pipe, to take part of the exponentials off
+// the MUFU unit (16 per clock per SM, as many as the tensor cores need for a
+// 128 x 128 x 128 tile pair).  Range reduction x = n + f with n = rint(x),
+// |f| <= 1/2, using the classic shifter: adding 1.5 * 2^23 rounds x to an
+// integer held in the low mantissa bits; 2^f by a degree-3 polynomial with
+// p(0) = 1 whose coefficients were fitted for this library by minimising the
+// maximum relative error on [-1/2, 1/2] (1.03e-4; P is then rounded to
+// 16 bits, a 2^-9 step); 2^n is added to the exponent field.  Valid for
+// x <= 127; x below -126 is clamped to -126 (2^-126 instead of a smaller
+// value), so callers use it only where no score is masked to -inf.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kShift = 12582912.f;   // 1.5 * 2^23
+    constexpr float c1 = 6.932791870e-01f, c2 = 2.422159912e-01f, c3 = 5.503048995e-02f;
+    x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+    const float2 j = __fadd2_rn(x, make_float2(kShift, kShift));
+    const float2 n = __fadd2_rn(j, make_float2(-kShift, -kShift));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+    q = __ffma2_rn(q, f, make_float2(c1, c1));
+    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+    // the low bits of j are n (two's complement); shifted by 23 they add n
+    // to the exponent of q (the shifter's own bits move out of the word)
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
