@@ -57,6 +57,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target oracle CPU time of the cpu_baseline sample")
     ap.add_argument("--flush-mib", type=int, default=512)
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="sweep workload only: Nq = Nk = N with B = max(1, 16384 // N)")
+    ap.add_argument("--causal", type=int, choices=[0, 1], default=None,
+                    help="override the workload's causal flag")
     return ap.parse_args(argv)
 
 
@@ -71,7 +75,17 @@ def load_peaks():
 
 def workload_cfg(args):
     from exact_attention_112_b200 import inputs
-    w = inputs.workload(args.workload, dtype=args.dtype)
+    over = {"dtype": args.dtype}
+    if args.seq_len is not None:
+        if args.workload != "sweep":
+            raise SystemExit("--seq-len applies to the sweep workload only")
+        over["N"] = args.seq_len
+    if args.causal is not None:
+        over["causal"] = bool(args.causal)
+    w = inputs.workload(args.workload, **over)
+    if args.seq_len is not None or args.causal is not None:
+        # keeps stored ncu traffic (keyed by workload name) off modified shapes
+        w["name"] = f"{w['name']}-N{w['Nq']}-{'causal' if w['causal'] else 'full'}"
     return w
 
 
