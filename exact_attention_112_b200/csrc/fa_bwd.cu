@@ -226,7 +226,7 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 // ---------------------------------------------------------------------------
 // 2. dK, dV for one 128-key tile per CTA.
 //
-// MMA issue order per query tile j (one thread, in-order tensor pipe):
+// MMA issue order per query tile j (one elected lane, in-order tensor pipe):
 //     dV(j)        once phase 1 of j has put P^T over the S^T columns
 //     S^T(j+1)
 //     dK(j)        once phase 2 of j has put dS^T over the dP^T columns

@@ -13,16 +13,20 @@
 // Q0, Q1 of one (batch, head)):
 //   * TMA streams Q once and K_j / V_j through a 2-stage shared-memory ring,
 //     handing each stage over with an mbarrier (expect_tx / complete_tx).
-//   * One thread issues tcgen05.mma: S_i = Q_i K_j^T (both operands from
-//     shared memory, fp32 accumulator in tensor memory) and O_i += P_i V_j
-//     (P_i read from tensor memory, V_j from shared memory).
+//   * The MMA warp issues tcgen05.mma from one elected lane while the whole
+//     warp runs the loop (warp-uniform descriptors and counters): S_i =
+//     Q_i K_j^T (both operands from shared memory, fp32 accumulator in tensor
+//     memory) and O_i += P_i V_j (P_i read from tensor memory, V_j from shared
+//     memory).
 //   * Two softmax warpgroups (one per Q tile, one thread per query row) read
 //     S_i from tensor memory, apply scale and mask in the base-2 domain
 //     (qk_scale = scale * log2(e), the constant derived in "Mastering
 //     FlashAttention: The Algebraic Foundation"), update the row max and sum in
 //     registers, write P_i back into the same tensor-memory columns as 16-bit
-//     values and signal the MMA thread.  While one warpgroup works on S_0 the
-//     tensor core computes S_1, and vice versa.
+//     values and signal the MMA warp.  While one warpgroup works on S_0 the
+//     tensor core computes S_1, and vice versa.  Three exponentials in four
+//     run on the MUFU unit, the fourth on the FMA pipe (exp2_fma2), so that
+//     the exponentials do not co-limit the loop with the tensor core.
 //   * Lazy rescale: the reference maximum m_ref of a row only moves when a new
 //     tile's maximum exceeds it by more than kTau (log2 units); only then are
 //     l and the O accumulator multiplied by alpha = 2^(m_ref_old - m_ref_new).
