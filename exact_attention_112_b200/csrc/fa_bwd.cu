@@ -257,8 +257,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     // ---- work unit: the key tiles that see the most query tiles come first
     const int BH = p.B * p.H;
-    const int t = blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    int t, bh;   // key tile 0 is seen by the most query tiles
+    unit_of(blockIdx.x, BH, (p.Nk + kBK - 1) / kBK, t, bh);
     const int kv0 = t * kBK;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
     int j_begin = 0;
@@ -645,8 +645,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ---- work unit: query tiles that see the most key tiles come first
     const int BH = p.B * p.H;
     const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
-    const int qt = (n_q_all - 1) - blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    int rank_, bh_;
+    unit_of(blockIdx.x, BH, n_q_all, rank_, bh_);
+    const int qt = (n_q_all - 1) - rank_;
+    const int bh = bh_;
     const int q0 = qt * kBQ;
     const int n_kv_all = (p.Nk + kBK - 1) / kBK;
     int n = n_kv_all;

@@ -66,4 +66,24 @@ cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D,
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,
                              cudaStream_t stream);
 
+// Work-unit order of the backward recompute kernels (one CTA = one unit):
+// heads in groups of kHeadGroup and, within a group, tile-major with the
+// heaviest tile rank first.  The CTAs in flight at any time then share the
+// streamed Q/dO (or K/V) tiles of a few heads in L2 instead of all heads',
+// and across the grid the long causal units still start before the short
+// ones.  Maps idx in [0, n_heads * n_tiles) one-to-one onto
+// (tile_rank, head); the caller turns tile_rank 0 into its heaviest tile.
+#ifdef __CUDACC__
+__device__ __forceinline__ void unit_of(int idx, int n_heads, int n_tiles, int &tile_rank, int &head) {
+    constexpr int kHeadGroup = 8;
+    const int per_group = kHeadGroup * n_tiles;
+    const int grp = idx / per_group;
+    const int r = idx - grp * per_group;
+    const int g0 = grp * kHeadGroup;
+    const int gsz = min(kHeadGroup, n_heads - g0);
+    tile_rank = r / gsz;
+    head = g0 + r % gsz;
+}
+#endif
+
 }  // namespace fa
