@@ -40,6 +40,13 @@ def test_many_tiles():
     check_backward(2, 3, 1024, 1024, 128, "bf16", True, seed=8)
 
 
+def test_head_groups_full_and_partial():
+    # 9 heads: one full group of 8 work units per tile rank and a partial
+    # group of 1, in both recompute kernels
+    check_backward(3, 3, 384, 384, 64, "bf16", True, seed=9)
+    check_backward(1, 9, 200, 330, 128, "f16", False, seed=10)
+
+
 def test_no_keys_and_no_queries():
     dev = torch.device("cuda")
     # Nk == 0: every output row empty, dQ = 0
