@@ -92,3 +92,60 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fa, "library_path", lambda: str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         fa.lib()
+
+
+def _bwd(L, dq=1, dk=1, ws=1, ws_bytes=1 << 20, B=1, H=1, Nq=128, Nk=128, D=64, causal=0,
+         scale=0.125, dtype=0, q=1):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    return L.fa_bwd(P(q), P(2), P(3), P(4), P(5), P(6), P(dq), P(dk), P(9), B, H, Nq, Nk, D,
+                    causal, ctypes.c_float(scale), dtype, None, P(ws), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_bwd_argument_errors_are_synchronous(L):
+    assert _bwd(L, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert _bwd(L, B=0) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, causal=3) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, dq=0) == fa.FA_ERR_INVALID_ARG          # null dQ with queries present
+    assert _bwd(L, dk=0) == fa.FA_ERR_INVALID_ARG          # null dK with keys present
+    assert _bwd(L, ws=0) == fa.FA_ERR_WORKSPACE            # no workspace
+    need = fa.fa_bwd_workspace_bytes(1, 1, 128, 128, 64)
+    assert _bwd(L, ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    # misaligned q
+    assert L.fa_bwd(ctypes.c_void_p(24), *[ctypes.c_void_p(16 * i) for i in range(2, 10)], 1, 1, 128,
+                    128, 64, 0, ctypes.c_float(0.1), 0, None, ctypes.c_void_p(16),
+                    ctypes.c_size_t(1 << 20), None) == fa.FA_ERR_INVALID_ARG
+
+
+def _split(L, num_splits=4, ws=1, ws_bytes=1 << 30, Nq=16, Nk=4096, D=128, k=1):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    return L.fa_fwd_splitkv(P(1), P(k), P(3), P(4), P(5), 1, 2, Nq, Nk, D, 0, ctypes.c_float(0.1),
+                            1, None, num_splits, P(ws), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_splitkv_argument_errors_are_synchronous(L):
+    assert _split(L, num_splits=0) == fa.FA_ERR_INVALID_ARG
+    assert _split(L, num_splits=257) == fa.FA_ERR_INVALID_ARG
+    assert _split(L, D=80) == fa.FA_ERR_UNSUPPORTED
+    assert _split(L, k=0) == fa.FA_ERR_INVALID_ARG
+    assert _split(L, ws=0) == fa.FA_ERR_WORKSPACE
+    need = fa.fa_fwd_splitkv_workspace_bytes(1, 2, 16, 4096, 128, 4)
+    assert _split(L, ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    assert _split(L, Nq=0, k=None, ws=None) == fa.FA_OK      # nothing to do, no CUDA call
+
+
+def test_splitkv_workspace_size(L):
+    # partial O (fp32) and partial LSE per row and split, each 256-byte aligned, + slack
+    rows = 1 * 2 * 16 * 4
+    need = fa.fa_fwd_splitkv_workspace_bytes(1, 2, 16, 4096, 128, 4)
+    assert need >= rows * 128 * 4 + rows * 4
+    assert need <= rows * 128 * 4 + rows * 4 + 3 * 256
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 2, 16, 4096, 128, 0) == 0
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 2, 16, 4096, 96, 4) == 0
+
+
+def test_noalloc_rejects_too_many_rows_before_any_cuda_call(L):
+    P = lambda x: ctypes.c_void_p(16 * x)
+    rows = fa.FA_BWD_NOALLOC_MAX_ROWS
+    assert L.fa_bwd_noalloc(*[P(i) for i in range(1, 10)], 1, 1, rows + 1, 128, 64, 0,
+                            ctypes.c_float(0.1), 0, None, None) == fa.FA_ERR_WORKSPACE
