@@ -19,7 +19,8 @@ Contents
     and the associative merge of the "twisted monoid" digest (setupai.cc,
     "Mastering FlashAttention: The Algebraic Foundation"), in float64.
 
-Array layout everywhere: ``[B, H, N, D]`` with D fastest; key bias ``[B, Nk]``.
+Array layout everywhere: ``[B, H, N, D]`` with D fastest; key bias ``[B, Nk]``;
+general additive mask ``[B or 1, H or 1, Nq, Nk]`` (or ``[Nq, Nk]``).
 """
 from __future__ import annotations
 
@@ -65,6 +66,17 @@ def _bind(lib):
                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                ip, ctypes.c_int, ip, ctypes.c_int, dp, dp, dp]
     lib.oracle_bwd.restype = None
+    L = ctypes.c_long
+    lib.oracle_fwd_mask.argtypes = [dp, dp, dp, dp, dp, L, L, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_double, ip,
+                                    ctypes.c_int, dp, dp]
+    lib.oracle_fwd_mask.restype = None
+    lib.oracle_bwd_mask.argtypes = [dp, dp, dp, dp, dp, L, L, dp, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                    ip, ctypes.c_int, ip, ctypes.c_int, dp, dp, dp]
+    lib.oracle_bwd_mask.restype = None
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -120,19 +132,37 @@ def default_scale(D: int) -> float:
     return 1.0 / np.sqrt(D)
 
 
+def _mask_arg(mask, B, H, Nq, Nk):
+    """(array, batch stride, head stride) for the C oracle; strides in
+    elements, 0 where the mask broadcasts over that axis."""
+    if mask is None:
+        return None, 0, 0
+    m = _f64(mask)
+    if m.ndim == 2:
+        m = m[None, None]
+    assert m.ndim == 4 and m.shape[2:] == (Nq, Nk), m.shape
+    assert m.shape[0] in (1, B) and m.shape[1] in (1, H), m.shape
+    assert not np.any(np.isposinf(m)) and not np.any(np.isnan(m)), "mask entries: finite or -inf"
+    hs = Nq * Nk if m.shape[1] == H and H > 1 else 0
+    bs = m.shape[1] * Nq * Nk if m.shape[0] == B and B > 1 else 0
+    return m, bs, hs
+
+
 class Oracle:
     """The oracle bound to one compiled copy of ``fa_oracle.c``."""
 
     def __init__(self, lib):
         self._lib = lib
 
-    def fwd(self, q, k, v, key_bias=None, causal=False, scale=None, rows=None):
+    def fwd(self, q, k, v, key_bias=None, causal=False, scale=None, rows=None, mask=None):
         """Exact attention forward in float64.
 
         q: [B,H,Nq,D]; k, v: [B,H,Nk,D]; key_bias: [B,Nk] or None (additive, after
-        scaling).  ``rows``: optional 1-D list of query-row indices evaluated for
-        every (b, h); None means all rows.  Returns ``(o, lse)`` with o
-        [B,H,R,D] and lse [B,H,R] (R = Nq or len(rows)).
+        scaling); mask: general additive mask [B or 1, H or 1, Nq, Nk] or
+        [Nq, Nk] (finite or -inf, added after scaling), or None.  ``rows``:
+        optional 1-D list of query-row indices evaluated for every (b, h); None
+        means all rows.  Returns ``(o, lse)`` with o [B,H,R,D] and lse [B,H,R]
+        (R = Nq or len(rows)).
         """
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, Nq, D = q.shape
@@ -153,21 +183,29 @@ class Oracle:
         lse = np.zeros((B, H, R), dtype=np.float64)
         if B * H * R == 0:
             return o, lse
-        self._lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, Nq, Nk, D,
-                           int(bool(causal)), float(scale),
-                           _ptr(rows_arr, ctypes.c_int), 0 if rows_arr is None else R,
-                           _ptr(o), _ptr(lse))
+        if mask is None:
+            self._lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, Nq, Nk, D,
+                               int(bool(causal)), float(scale),
+                               _ptr(rows_arr, ctypes.c_int), 0 if rows_arr is None else R,
+                               _ptr(o), _ptr(lse))
+        else:
+            m, bs, hs = _mask_arg(mask, B, H, Nq, Nk)
+            self._lib.oracle_fwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(m), bs, hs,
+                                    B, H, Nq, Nk, D, int(bool(causal)), float(scale),
+                                    _ptr(rows_arr, ctypes.c_int), 0 if rows_arr is None else R,
+                                    _ptr(o), _ptr(lse))
         return o, lse
 
 
     def bwd(self, q, k, v, dO, key_bias=None, causal=False, scale=None, bh_list=None,
-            rows=None):
+            rows=None, mask=None):
         """Exact gradients of L = sum(O * dO) w.r.t. q, k, v in float64.
 
         ``bh_list``: flat (b*H + h) indices to evaluate (None = all).  Returns
         ``(dq, dk, dv)`` of shapes [n, Nq, D], [n, Nk, D], [n, Nk, D].
         ``rows``: optional query-row subset; only those rows contribute (a
         bounded sample of the work for timing; None = the full gradient).
+        ``mask``: as in ``fwd``; it receives no gradient.
         """
         q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
         B, H, Nq, D = q.shape
@@ -189,11 +227,20 @@ class Oracle:
         dv = np.zeros((n, Nk, D))
         if n == 0:
             return dq, dk, dv
-        self._lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(dO), B, H, Nq,
-                           Nk, D, int(bool(causal)), float(scale),
-                           _ptr(bh, ctypes.c_int), n, _ptr(rows_arr, ctypes.c_int),
-                           0 if rows_arr is None else rows_arr.size,
-                           _ptr(dq), _ptr(dk), _ptr(dv))
+        if mask is None:
+            self._lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(dO), B, H, Nq,
+                               Nk, D, int(bool(causal)), float(scale),
+                               _ptr(bh, ctypes.c_int), n, _ptr(rows_arr, ctypes.c_int),
+                               0 if rows_arr is None else rows_arr.size,
+                               _ptr(dq), _ptr(dk), _ptr(dv))
+        else:
+            m, bs, hs = _mask_arg(mask, B, H, Nq, Nk)
+            self._lib.oracle_bwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(m), bs, hs,
+                                    _ptr(dO), B, H, Nq, Nk, D, int(bool(causal)),
+                                    float(scale), _ptr(bh, ctypes.c_int), n,
+                                    _ptr(rows_arr, ctypes.c_int),
+                                    0 if rows_arr is None else rows_arr.size,
+                                    _ptr(dq), _ptr(dk), _ptr(dv))
         return dq, dk, dv
 
 

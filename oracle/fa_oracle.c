@@ -23,8 +23,10 @@
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - mask = causal (bottom-right aligned: key j visible to query i iff
- *     j <= i + (Nk - Nq)) and/or an additive per-key bias [B, Nk] added after
- *     scaling; -inf entries give probability 0;
+ *     j <= i + (Nk - Nq)) and/or an additive per-key bias [B, Nk] and/or a
+ *     general additive mask M [B or 1, H or 1, Nq, Nk] (the "+ mask" of the
+ *     SDPA formula in full), both added after scaling; -inf entries give
+ *     probability 0;
  *   - a row with no visible key has O = 0 and LSE = -inf;
  *   - LSE is the natural log of sum_j exp(S_ij) over visible keys.
  *
@@ -52,8 +54,9 @@ static int key_visible(long i, long j, long Nq, long Nk, int causal)
  * S row).  Writes P_ij (normalised) into p_row[0..Nk) and returns LSE_i;
  * a row with no visible key gets P = 0 and LSE = -inf. */
 static double softmax_row(const double *qi, const double *kh,
-                          const double *bias_b, long i, long Nq, long Nk, long D,
-                          int causal, double scale, double *p_row)
+                          const double *bias_b, const double *mask_bh, long i,
+                          long Nq, long Nk, long D, int causal, double scale,
+                          double *p_row)
 {
     double m = -INFINITY;
     for (long j = 0; j < Nk; ++j) {
@@ -65,6 +68,7 @@ static double softmax_row(const double *qi, const double *kh,
             for (long d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
             s = scale * dot;
             if (bias_b) s += bias_b[j];
+            if (mask_bh) s += mask_bh[i * Nk + j];
         }
         p_row[j] = s;
         if (s > m) m = s;
@@ -85,11 +89,11 @@ static double softmax_row(const double *qi, const double *kh,
 
 /* One query row: O_i = sum_j P_ij V_j and LSE_i. */
 static void attn_row(const double *qi, const double *kh, const double *vh,
-                     const double *bias_b, long i, long Nq, long Nk, long D,
-                     int causal, double scale, double *p_row, double *o_i,
-                     double *lse_i)
+                     const double *bias_b, const double *mask_bh, long i, long Nq,
+                     long Nk, long D, int causal, double scale, double *p_row,
+                     double *o_i, double *lse_i)
 {
-    *lse_i = softmax_row(qi, kh, bias_b, i, Nq, Nk, D, causal, scale, p_row);
+    *lse_i = softmax_row(qi, kh, bias_b, mask_bh, i, Nq, Nk, D, causal, scale, p_row);
     for (long d = 0; d < D; ++d) o_i[d] = 0.0;
     for (long j = 0; j < Nk; ++j) {
         if (p_row[j] == 0.0) continue;
@@ -98,14 +102,18 @@ static void attn_row(const double *qi, const double *kh, const double *vh,
 }
 
 /*
- * Forward.  rows == NULL computes every query row; otherwise the nrows listed
- * row indices (each in [0, Nq)) of every (b, h).  Output o is
- * [B, H, nrows_eff, D] and lse [B, H, nrows_eff] in float64.
+ * Forward with a general additive mask.  mask == NULL means none; otherwise
+ * entry (b, h, i, j) is mask[b * mask_bstride + h * mask_hstride + i * Nk + j]
+ * (strides in elements; 0 broadcasts over that axis).  rows == NULL computes
+ * every query row; otherwise the nrows listed row indices (each in [0, Nq)) of
+ * every (b, h).  Output o is [B, H, nrows_eff, D] and lse [B, H, nrows_eff] in
+ * float64.
  */
-void oracle_fwd(const double *q, const double *k, const double *v,
-                const double *key_bias, int B, int H, int Nq, int Nk, int D,
-                int causal, double scale, const int *rows, int nrows,
-                double *o, double *lse)
+void oracle_fwd_mask(const double *q, const double *k, const double *v,
+                     const double *key_bias, const double *mask, long mask_bstride,
+                     long mask_hstride, int B, int H, int Nq, int Nk, int D,
+                     int causal, double scale, const int *rows, int nrows,
+                     double *o, double *lse)
 {
     long nr = rows ? nrows : Nq;
     long BH = (long)B * H;
@@ -119,9 +127,10 @@ void oracle_fwd(const double *q, const double *k, const double *v,
             const double *kh = k + bh * (long)Nk * D;
             const double *vh = v + bh * (long)Nk * D;
             const double *bias_b = key_bias ? key_bias + b * (long)Nk : NULL;
+            const double *mask_bh = mask ? mask + b * mask_bstride + (bh % H) * mask_hstride : NULL;
             for (long r = 0; r < nr; ++r) {
                 long i = rows ? rows[r] : r;
-                attn_row(qh + i * D, kh, vh, bias_b, i, Nq, Nk, D, causal,
+                attn_row(qh + i * D, kh, vh, bias_b, mask_bh, i, Nq, Nk, D, causal,
                          scale, s_row, o + (bh * nr + r) * D, lse + bh * nr + r);
             }
         }
@@ -129,8 +138,19 @@ void oracle_fwd(const double *q, const double *k, const double *v,
     }
 }
 
+/* Forward without a general mask (causal and per-key bias only). */
+void oracle_fwd(const double *q, const double *k, const double *v,
+                const double *key_bias, int B, int H, int Nq, int Nk, int D,
+                int causal, double scale, const int *rows, int nrows,
+                double *o, double *lse)
+{
+    oracle_fwd_mask(q, k, v, key_bias, NULL, 0, 0, B, H, Nq, Nk, D, causal, scale,
+                    rows, nrows, o, lse);
+}
+
 /*
- * Backward for a list of (b, h) pairs (bh_list[t] = b * H + h), full gradients.
+ * Backward for a list of (b, h) pairs (bh_list[t] = b * H + h), full gradients,
+ * with the general mask addressed as in oracle_fwd_mask (NULL = none).
  * Outputs dq [n_bh, Nq, D], dk and dv [n_bh, Nk, D] in float64.
  * Row by row: materialise P_i and dP_i, form dS_i, accumulate the three
  * gradients.  No stored O or LSE is used: both are recomputed from scratch.
@@ -138,11 +158,12 @@ void oracle_fwd(const double *q, const double *k, const double *v,
  * rows contribute (their dQ rows are exact, dK and dV hold only their share):
  * a bounded sample of the same work, used for CPU timing.
  */
-void oracle_bwd(const double *q, const double *k, const double *v,
-                const double *key_bias, const double *dO, int B, int H, int Nq,
-                int Nk, int D, int causal, double scale, const int *bh_list,
-                int n_bh, const int *q_rows, int n_q_rows, double *dq, double *dk,
-                double *dv)
+void oracle_bwd_mask(const double *q, const double *k, const double *v,
+                     const double *key_bias, const double *mask, long mask_bstride,
+                     long mask_hstride, const double *dO, int B, int H, int Nq,
+                     int Nk, int D, int causal, double scale, const int *bh_list,
+                     int n_bh, const int *q_rows, int n_q_rows, double *dq,
+                     double *dk, double *dv)
 {
     (void)B;
 #pragma omp parallel
@@ -158,6 +179,7 @@ void oracle_bwd(const double *q, const double *k, const double *v,
             const double *vh = v + bh * (long)Nk * D;
             const double *doh = dO + bh * (long)Nq * D;
             const double *bias_b = key_bias ? key_bias + b * (long)Nk : NULL;
+            const double *mask_bh = mask ? mask + b * mask_bstride + (bh % H) * mask_hstride : NULL;
             double *dqh = dq + t * (long)Nq * D;
             double *dkh = dk + t * (long)Nk * D;
             double *dvh = dv + t * (long)Nk * D;
@@ -168,8 +190,8 @@ void oracle_bwd(const double *q, const double *k, const double *v,
             for (long r = 0; r < n_rows; ++r) {
                 long i = q_rows ? q_rows[r] : r;
                 /* P_i: the softmax row, rebuilt from scratch */
-                double lse = softmax_row(qh + i * D, kh, bias_b, i, Nq, Nk, D,
-                                         causal, scale, p);
+                double lse = softmax_row(qh + i * D, kh, bias_b, mask_bh, i, Nq, Nk,
+                                         D, causal, scale, p);
                 if (lse == -INFINITY) continue;   /* no visible key: no gradient */
                 /* dP_ij = dO_i . V_j ;  Di = sum_j P_ij dP_ij */
                 double Di = 0.0;
@@ -193,6 +215,17 @@ void oracle_bwd(const double *q, const double *k, const double *v,
         free(p);
         free(dp);
     }
+}
+
+/* Backward without a general mask (causal and per-key bias only). */
+void oracle_bwd(const double *q, const double *k, const double *v,
+                const double *key_bias, const double *dO, int B, int H, int Nq,
+                int Nk, int D, int causal, double scale, const int *bh_list,
+                int n_bh, const int *q_rows, int n_q_rows, double *dq, double *dk,
+                double *dv)
+{
+    oracle_bwd_mask(q, k, v, key_bias, NULL, 0, 0, dO, B, H, Nq, Nk, D, causal,
+                    scale, bh_list, n_bh, q_rows, n_q_rows, dq, dk, dv);
 }
 
 /* Thread control for timing runs (OpenMP over (b, h) pairs). */

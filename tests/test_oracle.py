@@ -316,9 +316,118 @@ def pin_autograd(orc):
     return worst <= 1e-10, worst
 
 
+# ---- the general additive mask [B or 1, H or 1, Nq, Nk] ----------------------
+
+def rand_mask(shape, frac_masked=0.25, std=1.0):
+    """Finite N(0, std^2) entries with a random share set to -inf; column 0 of
+    every row stays finite so that no row is empty."""
+    m = RNG.standard_normal(shape) * std
+    m[RNG.random(shape) < frac_masked] = -np.inf
+    m[..., 0] = RNG.standard_normal(shape[:-1])
+    return m
+
+
+def pin_mask_library(orc):
+    """General mask: O == torch SDPA (float64) with the same additive float
+    mask, for full, head-broadcast and batch-broadcast shapes, also combined
+    with causal and a key bias."""
+    worst = 0.0
+    for (Nq, Nk, D, mshape, causal, wb) in [(9, 13, 5, (2, 3), False, False),
+                                            (9, 13, 5, (1, 3), False, True),
+                                            (11, 11, 8, (2, 1), True, False),
+                                            (7, 16, 4, (1, 1), False, False)]:
+        q, k, v, bias = rand_case(2, 3, Nq, Nk, D, causal, wb)
+        m = rand_mask(mshape + (Nq, Nk))
+        if causal:
+            m[..., :, 0] = 0.0
+        scale = 1.0 / math.sqrt(D)
+        o, _ = orc.fwd(q, k, v, bias, causal, scale, mask=m)
+        full = np.broadcast_to(m, (2, 3, Nq, Nk)).copy()
+        if causal:
+            full[:, :, ~visible_mask(Nq, Nk, True)] = -np.inf
+        if bias is not None:
+            full = full + bias[:, None, None, :]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            *(torch.tensor(x) for x in (q, k, v)), attn_mask=torch.tensor(full), scale=scale)
+        worst = max(worst, float(np.abs(o - ref.numpy()).max()))
+    return worst <= 1e-12, worst
+
+
+def pin_mask_row_shift(orc):
+    """Adding c_i to every entry of mask row i leaves O unchanged and adds c_i
+    to LSE_i (softmax is shift invariant per row); a mask applied to the wrong
+    axis or scaled would break this."""
+    q, k, v, _ = rand_case(2, 2, 10, 14, 6, False, False)
+    m = rand_mask((2, 2, 10, 14))
+    c = RNG.uniform(-5, 5, size=(2, 2, 10, 1))
+    o0, l0 = orc.fwd(q, k, v, None, False, 0.4, mask=m)
+    o1, l1 = orc.fwd(q, k, v, None, False, 0.4, mask=m + c)
+    err = max(float(np.abs(o1 - o0).max()), float(np.abs(l1 - (l0 + c[..., 0])).max()))
+    return err <= 1e-11, err
+
+
+def pin_mask_prefix_mean(orc):
+    """Q = 0 and a 0/-inf mask: O_i is the mean of the V rows the mask leaves
+    visible to row i and LSE_i = ln(#visible) (exact row/column indexing)."""
+    B, H, Nq, Nk, D = 1, 2, 12, 9, 4
+    q = np.zeros((B, H, Nq, D))
+    _, k, v, _ = rand_case(B, H, Nq, Nk, D, False, False)
+    vis = RNG.random((B, H, Nq, Nk)) < 0.5
+    vis[..., RNG.integers(0, Nk, size=(B, H, Nq))[..., None] == np.arange(Nk)] = True
+    m = np.where(vis, 0.0, -np.inf)
+    o, lse = orc.fwd(q, k, v, None, False, 1.0, mask=m)
+    err = 0.0
+    for h in range(H):
+        for i in range(Nq):
+            sel = vis[0, h, i]
+            want = v[0, h, sel].mean(axis=0)
+            err = max(err, float(np.abs(o[0, h, i] - want).max()),
+                      abs(float(lse[0, h, i]) - math.log(int(sel.sum()))))
+    return err <= 1e-12, err
+
+
+def pin_mask_causal_equivalence(orc):
+    """A 0/-inf mask holding the bottom-right causal pattern gives the causal
+    result (Nq != Nk both ways), forward and backward."""
+    err = 0.0
+    for (Nq, Nk) in [(7, 12), (12, 7)]:
+        q, k, v, _ = rand_case(1, 2, Nq, Nk, 5, True, False)
+        do = RNG.standard_normal(q.shape)
+        m = np.where(visible_mask(Nq, Nk, True), 0.0, -np.inf)
+        o0, l0 = orc.fwd(q, k, v, None, True, 0.5)
+        o1, l1 = orc.fwd(q, k, v, None, False, 0.5, mask=m)
+        g0 = orc.bwd(q, k, v, do, None, True, 0.5)
+        g1 = orc.bwd(q, k, v, do, None, False, 0.5, mask=m)
+        both = np.isfinite(l0)
+        empty_ok = bool(np.all(np.isneginf(l1[~both]))) and bool(np.all(np.isneginf(l0[~both])))
+        err = max(err, float(np.abs(o1 - o0).max()), float(np.abs(l1[both] - l0[both]).max()),
+                  0.0 if empty_ok else 1.0,
+                  *(float(np.abs(a - b).max()) for a, b in zip(g0, g1)))
+    return err <= 1e-12, err
+
+
+def pin_mask_autograd(orc):
+    """Backward with a general mask == torch autograd through float64 SDPA."""
+    q, k, v, _ = rand_case(2, 2, 9, 11, 6, False, False)
+    m = rand_mask((1, 2, 9, 11))
+    do = RNG.standard_normal(q.shape)
+    dq, dk, dv = orc.bwd(q, k, v, do, None, False, 0.35, mask=m)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.tensor(m),
+                                                           scale=0.35)
+    out.backward(torch.tensor(do))
+    worst = 0.0
+    for g, t in ((dq, tq), (dk, tk), (dv, tv)):
+        ref = t.grad.numpy().reshape(g.shape)
+        worst = max(worst, float(np.abs(g - ref).max()) / max(1e-30, float(np.abs(ref).max())))
+    return worst <= 1e-10, worst
+
+
 PINS = [pin_library, pin_uniform, pin_one_hot, pin_shift_invariance,
         pin_single_key, pin_brute,
-        pin_online, pin_finite_differences, pin_autograd]
+        pin_online, pin_finite_differences, pin_autograd,
+        pin_mask_library, pin_mask_row_shift, pin_mask_prefix_mean,
+        pin_mask_causal_equivalence, pin_mask_autograd]
 
 
 @pytest.fixture(scope="module")
@@ -432,6 +541,12 @@ MUTANTS = {
                        "dvh[j * D + d] += ds * doh[i * D + d];"),
     "bwd_dq_uses_v": ("dqh[i * D + d] += scale * ds * kh[j * D + d];",
                       "dqh[i * D + d] += scale * ds * vh[j * D + d];"),
+    "mask_dropped": ("if (mask_bh) s += mask_bh[i * Nk + j];", ""),
+    "mask_scaled": ("if (mask_bh) s += mask_bh[i * Nk + j];",
+                    "if (mask_bh) s += scale * mask_bh[i * Nk + j];"),
+    "mask_rows_reversed": ("if (mask_bh) s += mask_bh[i * Nk + j];",
+                           "if (mask_bh) s += mask_bh[(Nq - 1 - i) * Nk + j];"),
+    "mask_head_stride_ignored": ("(bh % H) * mask_hstride", "0 * mask_hstride"),
 }
 
 
