@@ -1,0 +1,90 @@
+"""The input recipe and the work counts, pinned to the figures the survey of
+the pages fixes (host only).
+
+FLOPs: 4*B*H*Nq*Nk*D per forward, halved when causal ("The same computation at
+real size" slide: 4*h*n^2*d_k for one Llama-3-8B layer), backward 2.5x.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_112_b200 import inputs, metrics
+
+
+def test_llama_layer_flops_match_the_slide():
+    # one non-causal Llama-3-8B layer: 4 * 32 * 8192^2 * 128 = 1.0995e12 (~1.1 TFLOP)
+    dense = metrics.fwd_flops(1, 32, 8192, 8192, 128, False)
+    assert dense == 4 * 32 * 8192 ** 2 * 128
+    assert abs(dense / 1e12 - 1.1) < 0.01
+    assert metrics.fwd_flops(1, 32, 8192, 8192, 128, True) == pytest.approx(5.50e11, rel=1e-3)
+
+
+@pytest.mark.parametrize("cfg,flops", [
+    (("tiny", {}), 1.68e7),
+    (("llama", {}), 5.50e11),
+    (("stress", {}), 2.75e11),
+    (("sweep", {"N": 512, "causal": False}), 6.87e10),
+    (("sweep", {"N": 16384, "causal": False}), 2.20e12),
+    (("sweep", {"N": 32768, "causal": False}), 8.80e12),
+])
+def test_config_flops(cfg, flops):
+    name, over = cfg
+    w = inputs.workload(name, **over)
+    f = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    assert f == pytest.approx(flops, rel=2e-3)
+
+
+def test_backward_config_flops():
+    w = inputs.workload("bwd")
+    f = metrics.bwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    assert f == pytest.approx(6.87e11, rel=2e-3)
+    assert f == 2.5 * metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+
+
+def test_llama_forward_bytes():
+    # Q, K, V, O: 4 x 64 MiB of 16-bit values, plus 1 MiB of fp32 LSE
+    b = metrics.fwd_bytes(1, 32, 8192, 8192, 128)
+    assert b == 4 * 64 * 2 ** 20 + 2 ** 20
+
+
+def test_sweep_batch_rule():
+    # B = max(1, 16384 // N): N = 32768 runs B = 1
+    for n, b in [(512, 32), (1024, 16), (8192, 2), (16384, 1), (32768, 1)]:
+        w = inputs.workload("sweep", N=n)
+        assert (w["B"], w["Nq"], w["Nk"]) == (b, n, n)
+
+
+def test_stress_bias_masks_205_distinct_keys_per_batch():
+    w = inputs.workload("stress")
+    inp = inputs.make_inputs(2, 1, 8, w["Nk"], 64, dtype="bf16", seed=w["seed"],
+                             bias_frac=w["bias_frac"])
+    bias = inp["key_bias"].numpy()
+    assert bias.shape == (2, 2048)
+    for b in range(2):
+        assert int(np.isneginf(bias[b]).sum()) == round(0.1 * 2048) == 205
+        assert np.all(bias[b][np.isfinite(bias[b])] == 0.0)
+    assert not np.array_equal(np.isneginf(bias[0]), np.isneginf(bias[1]))
+
+
+def test_inputs_are_seeded_and_rounded_once():
+    a = inputs.make_inputs(1, 2, 33, 17, 64, dtype="bf16", seed=5, with_dO=True)
+    b = inputs.make_inputs(1, 2, 33, 17, 64, dtype="bf16", seed=5, with_dO=True)
+    c = inputs.make_inputs(1, 2, 33, 17, 64, dtype="bf16", seed=6, with_dO=True)
+    for key in ("q", "k", "v", "do"):
+        assert a[key].dtype == torch.bfloat16
+        assert torch.equal(a[key], b[key])
+    assert not torch.equal(a["q"], c["q"])
+    # the oracle receives exactly the rounded values
+    q64 = inputs.to_f64(a["q"])
+    assert np.array_equal(q64, a["q"].to(torch.float64).numpy())
+    assert np.array_equal(q64.astype(np.float32), q64)
+
+
+def test_sample_rows_cover_every_tile_boundary():
+    rows = inputs.sample_rows(1000, seed=3)
+    for t in range(0, 1000, 128):
+        assert t in rows and min(t + 127, 999) in rows
+    assert rows[0] == 0 and rows[-1] == 999
+    assert np.all(np.diff(rows) > 0)
