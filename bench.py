@@ -61,6 +61,11 @@ def parse_args(argv=None):
                     help="sweep workload only: Nq = Nk = N with B = max(1, 16384 // N)")
     ap.add_argument("--causal", type=int, choices=[0, 1], default=None,
                     help="override the workload's causal flag")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (smaller profiling cases)")
+    ap.add_argument("--splits", type=int, default=None,
+                    help="forward through fa_fwd_splitkv with this many key ranges "
+                         "(default 16 for the decode workload, else the single-pass fa_fwd)")
     return ap.parse_args(argv)
 
 
@@ -82,10 +87,13 @@ def workload_cfg(args):
         over["N"] = args.seq_len
     if args.causal is not None:
         over["causal"] = bool(args.causal)
+    if args.heads is not None:
+        over["H"] = args.heads
     w = inputs.workload(args.workload, **over)
-    if args.seq_len is not None or args.causal is not None:
+    if args.seq_len is not None or args.causal is not None or args.heads is not None:
         # keeps stored ncu traffic (keyed by workload name) off modified shapes
-        w["name"] = f"{w['name']}-N{w['Nq']}-{'causal' if w['causal'] else 'full'}"
+        w["name"] = f"{w['name']}-H{w['H']}-N{w['Nq']}-{'causal' if w['causal'] else 'full'}"
+    w["splits"] = args.splits if args.splits is not None else (16 if args.workload == "decode" else 1)
     return w
 
 
@@ -101,7 +109,7 @@ def flops_of(w, passes):
 
 WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention backward workload",
                    "tiny": "tiny attention", "stress": "numerical-stress attention",
-                   "sweep": "sequence-sweep attention"}
+                   "sweep": "sequence-sweep attention", "decode": "split-KV decode attention"}
 
 
 # Algorithmic FLOPs of one launch of each kernel, as multiples of the forward's
@@ -111,10 +119,12 @@ WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention back
 # (0.5x forward) plus a recomputation of S and dP that is not algorithmic work.
 # When both run as one launch (fa_bwd_grad_kernel) it does all five products
 # (2.5x forward) and executes seven (3.5x).
-KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5,
+KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_fwd_split_kernel": 1.0,
+                       "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5,
                        "fa_bwd_grad_kernel": 2.5}
 # tile products each kernel executes, as multiples of the forward (2 products)
-KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5,
+KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_fwd_split_kernel": 1.0,
+                        "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5,
                         "fa_bwd_grad_kernel": 3.5}
 
 
@@ -158,7 +168,8 @@ def kernel_table(records, w):
 def workload_name(w, passes):
     return (f"{WORKLOAD_TITLES.get(w['name'], w['name'])} {'+'.join(passes)}: B={w['B']} H={w['H']} "
             f"Nq={w['Nq']} Nk={w['Nk']} D={w['D']} "
-            f"{'causal' if w['causal'] else 'non-causal'} {w['dtype']}")
+            f"{'causal' if w['causal'] else 'non-causal'} {w['dtype']}"
+            + (f", keys in {w['splits']} split-KV ranges" if w.get("splits", 1) > 1 else ""))
 
 
 # --------------------------------------------------------------------------
@@ -230,19 +241,26 @@ def oracle_sample_setup(w, passes):
     return {k: f(inp[k]) for k in ("q", "k", "v", "key_bias", "do")}
 
 
-def oracle_rows_time(arrs, w, rows, passes):
+def oracle_rows_time(arrs, w, rows, passes, outputs=None):
     """Run the oracle's passes on the query rows `rows` of every (b, h); return
-    (seconds, algorithmic FLOPs of that share of the step)."""
+    (seconds, algorithmic FLOPs of that share of the step).  If `outputs` is a
+    dict, the oracle's results are stored in it: o, lse of those rows and the
+    exact dQ of those rows (the row-sampled backward's dK, dV hold only the
+    sampled rows' share and are not kept)."""
     import numpy as np
     import oracle
     scale = 1.0 / math.sqrt(w["D"])
     t0 = time.perf_counter()
     if "fwd" in passes:
-        oracle.fwd(arrs["q"], arrs["k"], arrs["v"], arrs["key_bias"], w["causal"], scale,
-                   rows=rows)
+        r = oracle.fwd(arrs["q"], arrs["k"], arrs["v"], arrs["key_bias"], w["causal"], scale,
+                       rows=rows)
+        if outputs is not None:
+            outputs["o"], outputs["lse"] = r
     if "bwd" in passes:
-        oracle.bwd(arrs["q"], arrs["k"], arrs["v"], arrs["do"], arrs["key_bias"], w["causal"],
-                   scale, rows=rows)
+        r = oracle.bwd(arrs["q"], arrs["k"], arrs["v"], arrs["do"], arrs["key_bias"], w["causal"],
+                       scale, rows=rows)
+        if outputs is not None:
+            outputs["dq"] = r[0][:, rows]
     dt = time.perf_counter() - t0
     rows = np.asarray(rows)
     if w["causal"]:
@@ -254,9 +272,62 @@ def oracle_rows_time(arrs, w, rows, passes):
     return dt, fl
 
 
-def pick_rows(w, n):
+def pick_rows(w, n, boundaries=False):
+    """n evenly spaced query rows (plus, with `boundaries`, the first and last
+    row of every 128-row tile), sorted and unique."""
     import numpy as np
-    return np.unique(np.linspace(0, w["Nq"] - 1, max(1, n)).round().astype(np.int64))
+    rows = np.linspace(0, w["Nq"] - 1, max(1, n)).round().astype(np.int64)
+    if boundaries:
+        t = np.arange(0, w["Nq"], 128)
+        rows = np.concatenate([rows, t, np.minimum(t + 127, w["Nq"] - 1)])
+    return np.unique(rows)
+
+
+# Acceptance bar of the GPU results against the float64 oracle (the same
+# figures the parity tests use): O max-abs error per storage type, LSE max-abs
+# error, and gradients max|g - g_ref| / max|g_ref|.
+TOL_O = {"f16": 1e-2, "bf16": 2e-2}
+TOL_LSE = 1e-3
+TOL_GRAD_REL = 5e-2
+
+
+def parity_report(w, rows, ref, gpu):
+    """Compare the GPU's outputs of the benchmarked configuration with the
+    oracle's on the sampled rows (O, LSE, dQ: each row depends only on its own
+    query and all keys, so the sample is exact for those rows), and check two
+    identities that hold at any size for dK and dV (per (b, h) and d):
+        sum_j dV_j = sum_i dO_i   over rows that see a key (sum_j P_ij = 1),
+        sum_j dK_j = 0            (sum_j dS_ij = D_i - D_i = 0).
+    Returns a dict with the errors and `ok`."""
+    import numpy as np
+    rep, ok = {"rows_per_head": int(len(rows)), "heads": w["B"] * w["H"]}, True
+    if "o" in ref:
+        o = gpu["o"][:, :, rows]
+        lse = gpu["lse"][:, :, rows]
+        fin = np.isfinite(ref["lse"])
+        same_empty = bool(np.array_equal(np.isfinite(lse), fin))
+        err_o = float(np.abs(o - ref["o"]).max())
+        err_l = float(np.abs(lse[fin] - ref["lse"][fin]).max()) if fin.any() else 0.0
+        rep.update(o_max_abs=err_o, lse_max_abs=err_l, empty_rows_match=same_empty)
+        ok &= same_empty and err_o <= TOL_O[w["dtype"]] and err_l <= TOL_LSE
+    if "dq" in ref:
+        g = gpu["dq"].reshape(w["B"] * w["H"], w["Nq"], w["D"])[:, rows]
+        err = float(np.abs(g - ref["dq"]).max() / max(np.abs(ref["dq"]).max(), 1e-30))
+        rep["dq_rel_to_max"] = err
+        ok &= err <= TOL_GRAD_REL
+        # identities for dK and dV (float64 sums of the 16-bit results)
+        vis = np.ones(w["Nq"], dtype=bool)
+        if w["causal"]:
+            vis = np.arange(w["Nq"]) + (w["Nk"] - w["Nq"]) >= 0
+        sum_do = gpu["do"][:, :, vis].sum(axis=2)
+        sum_dv = gpu["dv"].sum(axis=2)
+        e_dv = float(np.abs(sum_dv - sum_do).max() / max(np.abs(sum_do).max(), 1e-30))
+        e_dk = float(np.abs(gpu["dk"].sum(axis=2)).max() /
+                     max(np.abs(gpu["dk"]).sum(axis=2).max(), 1e-30))
+        rep.update(sum_dv_rel=e_dv, sum_dk_rel=e_dk)
+        ok &= e_dv <= 1e-2 and e_dk <= 1e-2
+    rep["ok"] = bool(ok)
+    return rep
 
 
 def sample_text(w, rows, passes):
@@ -264,17 +335,28 @@ def sample_text(w, rows, passes):
             f"each of the {w['B'] * w['H']} (b,h) pairs")
 
 
-def cpu_baseline(w, target_s, passes):
+def cpu_baseline(w, target_s, passes, gpu=None):
+    """Time the oracle on a bounded row sample of the workload.  With `gpu`
+    (host copies of the GPU's outputs for the same inputs), its results on that
+    sample are also the parity check of the benchmarked run; returns
+    (baseline, parity report or None)."""
     import oracle
     arrs = oracle_sample_setup(w, passes)
     cores = oracle.max_threads()
     dt, fl = oracle_rows_time(arrs, w, pick_rows(w, 8), passes)          # calibration
     n = max(8, int(8 * target_s / max(dt, 1e-3)))
-    rows = pick_rows(w, min(n, w["Nq"]))
-    dt, fl = oracle_rows_time(arrs, w, rows, passes)
-    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+    rows = pick_rows(w, min(n, w["Nq"]), boundaries=gpu is not None)
+    ref = {}
+    dt, fl = oracle_rows_time(arrs, w, rows, passes, outputs=ref)
+    base = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": sample_text(w, rows, passes) + f" ({fl / 1e9:.1f} GFLOP algorithmic, {dt:.1f} s)",
             "seconds": dt}
+    if gpu is None:
+        return base, None
+    gpu = dict(gpu)
+    if "bwd" in passes:
+        gpu["do"] = arrs["do"]
+    return base, parity_report(w, rows, ref, gpu)
 
 
 def run_reference(args):
@@ -351,10 +433,22 @@ def run_ours(args):
     flush = torch.empty(args.flush_mib * (1 << 20), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    splits = w["splits"]
+    if splits > 1:
+        ws_split = torch.empty(fa.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, splits),
+                               dtype=torch.uint8, device=dev)
+
+    def forward():
+        if splits > 1:
+            fa.fa_fwd_splitkv(q, k, v, o, lse, splits, ws_split, causal=causal, key_bias=bias,
+                              stream=stream)
+        else:
+            fa.fa_fwd(q, k, v, o, lse, causal=causal, key_bias=bias, stream=stream)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        fa.fa_fwd(q, k, v, o, lse, causal=causal, key_bias=bias, stream=stream)
+        forward()
         if ev is not None:
             ev[1].record(stream)
         if "bwd" in passes:
@@ -368,6 +462,20 @@ def run_ours(args):
         step()
     torch.cuda.synchronize(dev)
     assert fa.fa_device_status(stream) == fa.FA_OK
+
+    # ---- before timing: the oracle on a row sample (the cpu_baseline leg),
+    # whose results also check the outputs of the warm-up steps above
+    cpu_line, parity = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gpu_out = {"o": o.float().cpu().numpy(), "lse": lse.cpu().numpy()}
+        if "bwd" in passes:
+            gpu_out.update({n_: t_.float().cpu().numpy() for n_, t_ in
+                            (("dq", dq), ("dk", dk), ("dv", dv))})
+        cpu_line, parity = cpu_baseline(w, args.cpu_seconds, passes, gpu_out)
+        if not parity["ok"]:
+            print(json.dumps({"error": "parity check against the oracle failed",
+                              "parity": parity}), file=sys.stderr, flush=True)
+            return 1
 
     n_ev = 3 if "bwd" in passes else 2
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
@@ -419,7 +527,7 @@ def run_ours(args):
         q.copy_(host["q"], non_blocking=True)
         k.copy_(host["k"], non_blocking=True)
         v.copy_(host["v"], non_blocking=True)
-        fa.fa_fwd(q, k, v, o, lse, causal=causal, key_bias=bias, stream=stream)
+        forward()
         out_o.copy_(o, non_blocking=True)
         out_lse.copy_(lse, non_blocking=True)
         if "bwd" in passes:
@@ -461,7 +569,7 @@ def run_ours(args):
         "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
         "config": {"workload": workload_name(w, passes), "B": B, "H": H, "Nq": Nq, "Nk": Nk,
-                   "D": D, "causal": causal, "passes": passes,
+                   "D": D, "causal": causal, "passes": passes, "kv_splits": splits,
                    "l2": f"flushed between steps ({args.flush_mib} MiB write, outside the events)",
                    "parallelism": "replicas" if world == 1 else f"{world} ranks, independent (b,h) shards"},
         "roofline": roof,
@@ -474,8 +582,9 @@ def run_ours(args):
                      for p in kern_ms},
         "kernels": kernels,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, passes)
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
+        line["parity"] = parity
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -492,19 +601,32 @@ def load_traffic(kernel, w):
     try:
         d = json.load(open(path))
         ent = d.get(f"{kernel}:{w['name']}")
-        if ent and ent.get("kernel_rev") == kernel_rev():
+        if ent and ent.get("kernel_rev") == kernel_rev(kernel):
             return ent["bytes_per_launch"]
     except (OSError, ValueError):
         pass
     return None
 
 
-def kernel_rev():
-    """Content hash of the CUDA sources, so stale ncu traffic is not reported."""
+# The source file that defines each kernel; its revision also covers the
+# device headers every kernel file includes.
+KERNEL_SOURCE = {"fa_fwd_kernel": "fa_fwd.cu", "fa_bwd_dkdv_kernel": "fa_bwd.cu",
+                 "fa_bwd_dq_kernel": "fa_bwd.cu", "fa_bwd_pre_kernel": "fa_bwd.cu"}
+DEVICE_HEADERS = ("fa_ptx.cuh", "fa_internal.h")
+
+
+def kernel_rev(kernel=None):
+    """Content hash of the CUDA sources a kernel is built from (its own .cu file
+    and the shared device headers; every source when the kernel is not known),
+    so that ncu traffic taken from an older build is not reported."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "exact_attention_112_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    names = sorted(os.listdir(csrc))
+    if kernel in KERNEL_SOURCE:
+        names = [n for n in names if n == KERNEL_SOURCE[kernel] or n in DEVICE_HEADERS]
+    for f in names:
+        h.update(f.encode())
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 

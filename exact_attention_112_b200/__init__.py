@@ -124,17 +124,74 @@ def _check(status, what):
         raise FaError(status, what)
 
 
+def _bad(what, msg):
+    raise FaError(FA_ERR_INVALID_ARG, f"{what}: {msg}")
+
+
+def _validate(what, q, k, v, *, o=None, lse=None, dO=None, dq=None, dk=None, dv=None,
+              key_bias=None, workspace=None, outputs=()):
+    """Check every tensor handed to the C ABI before its pointer is taken.
+
+    The library sees only pointers and the sizes derived from ``q`` and ``k``,
+    so a tensor of the wrong shape, dtype, layout or device would make the
+    kernels read or write outside its allocation.  Checked here: q is
+    [B,H,Nq,D] f16/bf16; k, v are [B,H,Nk,D] of q's dtype; o, dO, dq have q's
+    shape and dtype; dk, dv have k's; lse is float32 [B,H,Nq]; key_bias is
+    float32 [B,Nk]; every tensor (workspace included) is contiguous and on the
+    current CUDA device.  Returns (B, H, Nq, Nk, D, dtype code).
+    """
+    import torch
+    if q is None or q.dim() != 4:
+        _bad(what, "q must be a 4-D tensor [B, H, Nq, D]")
+    code = _dtype_code(q)
+    B, H, Nq, D = q.shape
+    if k is None or v is None:
+        _bad(what, "k and v are required")
+    if k.dim() != 4 or tuple(k.shape[:2]) != (B, H) or k.shape[3] != D:
+        _bad(what, f"k must be [B={B}, H={H}, Nk, D={D}], got {tuple(k.shape)}")
+    Nk = k.shape[2]
+    want = {"q": (q, (B, H, Nq, D), q.dtype), "k": (k, (B, H, Nk, D), q.dtype),
+            "v": (v, (B, H, Nk, D), q.dtype)}
+    for name, t, shape, dt in (("o", o, (B, H, Nq, D), q.dtype),
+                               ("lse", lse, (B, H, Nq), torch.float32),
+                               ("dO", dO, (B, H, Nq, D), q.dtype),
+                               ("dq", dq, (B, H, Nq, D), q.dtype),
+                               ("dk", dk, (B, H, Nk, D), q.dtype),
+                               ("dv", dv, (B, H, Nk, D), q.dtype),
+                               ("key_bias", key_bias, (B, Nk), torch.float32)):
+        if t is not None:
+            want[name] = (t, shape, dt)
+        elif name in outputs:
+            _bad(what, f"{name} is required")
+    for name, (t, shape, dt) in want.items():
+        if tuple(t.shape) != shape:
+            _bad(what, f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        if t.dtype != dt:
+            _bad(what, f"{name} must be {dt}, got {t.dtype}")
+    tensors = [t for t, _, _ in want.values()]
+    if workspace is not None:
+        tensors.append(workspace)
+    for t in tensors:
+        if not t.is_contiguous():
+            _bad(what, "every tensor must be contiguous")
+    for t in tensors:
+        if not t.is_cuda:
+            _bad(what, f"every tensor must be on a CUDA device, got {t.device}")
+    dev = torch.cuda.current_device()
+    for t in tensors:
+        if t.device.index != dev:
+            _bad(what, f"every tensor must be on the current device cuda:{dev}, got {t.device}")
+    return B, H, Nq, Nk, D, code
+
+
 def fa_fwd(q, k, v, o, lse, causal=False, scale=None, key_bias=None, stream=None):
     """Forward pass into caller-owned ``o`` [B,H,Nq,D] and ``lse`` [B,H,Nq] fp32."""
-    B, H, Nq, D = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, D, code = _validate("fa_fwd", q, k, v, o=o, lse=lse, key_bias=key_bias,
+                                      outputs=("o", "lse"))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    for t in (q, k, v, o, lse) + (() if key_bias is None else (key_bias,)):
-        if not t.is_contiguous():
-            raise FaError(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be contiguous")
     st = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
-                      int(bool(causal)), float(scale), _dtype_code(q), _ptr(key_bias),
+                      int(bool(causal)), float(scale), code, _ptr(key_bias),
                       _stream_ptr(stream))
     _check(st, "fa_fwd")
 
@@ -147,13 +204,14 @@ def fa_fwd_splitkv(q, k, v, o, lse, num_splits, workspace, causal=False, scale=N
                    key_bias=None, stream=None):
     """Split-KV forward (few queries, many keys) into caller-owned o, lse,
     with a caller-owned workspace of fa_fwd_splitkv_workspace_bytes() bytes."""
-    B, H, Nq, D = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, D, code = _validate("fa_fwd_splitkv", q, k, v, o=o, lse=lse,
+                                      key_bias=key_bias, workspace=workspace,
+                                      outputs=("o", "lse"))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     nbytes = workspace.numel() * workspace.element_size()
     st = lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
-                              int(bool(causal)), float(scale), _dtype_code(q), _ptr(key_bias),
+                              int(bool(causal)), float(scale), code, _ptr(key_bias),
                               int(num_splits), _ptr(workspace), nbytes, _stream_ptr(stream))
     _check(st, "fa_fwd_splitkv")
 
@@ -165,19 +223,32 @@ def fa_bwd_workspace_bytes(B, H, Nq, Nk, D) -> int:
 def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, causal=False, scale=None,
            key_bias=None, stream=None):
     """Backward pass into caller-owned dq, dk, dv, using a caller-owned workspace."""
-    B, H, Nq, D = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, D, code = _validate("fa_bwd", q, k, v, o=o, lse=lse, dO=dO, dq=dq, dk=dk,
+                                      dv=dv, key_bias=key_bias, workspace=workspace,
+                                      outputs=("o", "lse", "dO", "dq", "dk", "dv"))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     nbytes = workspace.numel() * workspace.element_size()
     st = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
                       _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)), float(scale),
-                      _dtype_code(q), _ptr(key_bias), _ptr(workspace), nbytes,
+                      code, _ptr(key_bias), _ptr(workspace), nbytes,
                       _stream_ptr(stream))
     _check(st, "fa_bwd")
 
 
-FA_BWD_NOALLOC_MAX_ROWS = 1048576
+def _header_define(name: str) -> int:
+    """Integer value of a ``#define`` in include/fa.h (the one source of the
+    library's compile-time limits)."""
+    import re
+    path = os.path.join(os.path.dirname(_HERE), "include", "fa.h")
+    with open(path) as f:
+        m = re.search(rf"^#define\s+{name}\s+(\d+)\s*$", f.read(), flags=re.M)
+    if m is None:
+        raise RuntimeError(f"{name} is not defined in {path}")
+    return int(m.group(1))
+
+
+FA_BWD_NOALLOC_MAX_ROWS = _header_define("FA_BWD_NOALLOC_MAX_ROWS")
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, causal=False, scale=None, key_bias=None,
@@ -185,13 +256,14 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, causal=False, scale=None, ke
     """Backward without a workspace, for callers that cannot allocate device
     memory (the scratch is a fixed array inside libfa.so; B*H*Nq must not
     exceed FA_BWD_NOALLOC_MAX_ROWS).  See include/fa.h."""
-    B, H, Nq, D = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, D, code = _validate("fa_bwd_noalloc", q, k, v, o=o, lse=lse, dO=dO, dq=dq,
+                                      dk=dk, dv=dv, key_bias=key_bias,
+                                      outputs=("o", "lse", "dO", "dq", "dk", "dv"))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     st = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
                               _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)),
-                              float(scale), _dtype_code(q), _ptr(key_bias), _stream_ptr(stream))
+                              float(scale), code, _ptr(key_bias), _stream_ptr(stream))
     _check(st, "fa_bwd_noalloc")
 
 

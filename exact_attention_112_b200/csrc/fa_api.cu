@@ -433,13 +433,19 @@ extern "C" int fa_bwd_noalloc(const void *q, const void *k, const void *v, const
                               const float *lse, const void *dO, void *dq, void *dk, void *dv, int B,
                               int H, int Nq, int Nk, int D, int causal, float scale, int dtype,
                               const float *key_bias, void *stream) {
-    // Too many query rows for the fixed scratch: refuse before touching the GPU.
-    if (B >= 1 && H >= 1 && Nq >= 0 &&
-        static_cast<long long>(B) * H * Nq > static_cast<long long>(kNoAllocMaxRows))
-        return FA_ERR_WORKSPACE;
-    int dev;
-    int st = current_device(&dev);
+    // Argument errors first, with the same codes as fa_bwd(); then the size
+    // limit of the fixed scratch; both before any CUDA call.
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
     if (st != FA_OK) return st;
+    if (static_cast<long long>(B) * H * Nq > static_cast<long long>(kNoAllocMaxRows))
+        return FA_ERR_WORKSPACE;
+    // The device must be usable (an sm_100 GPU) before the scratch array's
+    // address is asked for: on any other device the library has no image and
+    // the lookup would fail with a less precise code.
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
     float *scratch = nullptr;
     if ((st = noalloc_scratch(dev, &scratch)) != FA_OK) return st;
     // Every scratch entry the kernels read is written earlier in the same call

@@ -17,6 +17,7 @@ d_k = 128, n = 8192; the 32k-context anecdote of the lastdictionary.com
           V ~ U(-1,1), -inf key bias on 205 (= round(0.1 * 2048)) seeded
           key columns per batch
   bwd     B=2  H=32 N=4096  D=128 bf16 causal, Q,K,V,dO ~ N(0,1)
+  decode  B=1  H=8  Nq=256 Nk=65536 D=128 bf16 non-causal (split-KV)  N(0,1)
 
 There is no public dataset behind these: i.i.d. activations of the named shapes
 stand in for a real layer's Q/K/V (no trained weights are needed or used).
@@ -50,6 +51,11 @@ def workload(name: str, **over) -> dict:
         "bwd": dict(B=2, H=32, Nq=4096, Nk=4096, D=128, dtype="bf16",
                     causal=True, qk_std=1.0, v_dist="normal", bias_frac=0.0,
                     seed=1004),
+        # few queries against a long key sequence (the shape the split-KV
+        # forward is for): 256 query rows of 8 heads over 65536 keys
+        "decode": dict(B=1, H=8, Nq=256, Nk=65536, D=128, dtype="bf16",
+                       causal=False, qk_std=1.0, v_dist="normal", bias_frac=0.0,
+                       seed=1005),
     }[name]
     cfg = dict(base)
     cfg.update(over)

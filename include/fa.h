@@ -45,7 +45,9 @@
  *             wait that exceeds its time limit makes the kernel give up
  *             cleanly and latch FA_ERR_DEVICE_TIMEOUT in a per-device error
  *             word, read and cleared by fa_device_status().
- * Threads     Calls on different streams may run concurrently.
+ * Threads     Calls on different streams may run concurrently, except
+ *             fa_bwd_noalloc(), whose calls all share one scratch array
+ *             (see its description below).
  */
 #ifndef FA_H
 #define FA_H
@@ -134,8 +136,9 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
  * the per-row scratch lives in a fixed array compiled into the library
  * (4 * FA_BWD_NOALLOC_MAX_ROWS bytes plus 256, held on every GPU that loads the
  * library until the process exits).  Nothing is allocated by this call.
- *   - B * H * Nq > FA_BWD_NOALLOC_MAX_ROWS returns FA_ERR_WORKSPACE before any
- *     GPU work.
+ *   - Argument errors are reported as by fa_bwd(); then
+ *     B * H * Nq > FA_BWD_NOALLOC_MAX_ROWS returns FA_ERR_WORKSPACE; both
+ *     before any CUDA call.
  *   - The first call on a device asks the CUDA runtime for the array's device
  *     address (cudaGetSymbolAddress); make that first call before any stream
  *     capture begins.

@@ -149,3 +149,109 @@ def test_noalloc_rejects_too_many_rows_before_any_cuda_call(L):
     rows = fa.FA_BWD_NOALLOC_MAX_ROWS
     assert L.fa_bwd_noalloc(*[P(i) for i in range(1, 10)], 1, 1, rows + 1, 128, 64, 0,
                             ctypes.c_float(0.1), 0, None, None) == fa.FA_ERR_WORKSPACE
+
+
+def test_noalloc_limit_matches_header_and_accepts_the_limit(L):
+    """The Python constant is read from include/fa.h; exactly MAX_ROWS rows is
+    not refused for size (an invalid dtype stops it at validation instead),
+    and argument errors come before the size check."""
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    m = re.search(r"^#define\s+FA_BWD_NOALLOC_MAX_ROWS\s+(\d+)\s*$", text, flags=re.M)
+    assert m and int(m.group(1)) == fa.FA_BWD_NOALLOC_MAX_ROWS
+    P = lambda x: ctypes.c_void_p(16 * x)
+    rows = fa.FA_BWD_NOALLOC_MAX_ROWS
+
+    def call(B, H, Nq, dtype=0, D=64, ptrs=True):
+        args = [P(i) for i in range(1, 10)] if ptrs else [None] * 9
+        return L.fa_bwd_noalloc(*args, B, H, Nq, 128, D, 0, ctypes.c_float(0.1), dtype, None, None)
+
+    assert call(1, 1, rows, dtype=7) == fa.FA_ERR_UNSUPPORTED
+    assert call(1, 16, rows // 16, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(1, 1, rows + 1, dtype=7) == fa.FA_ERR_UNSUPPORTED   # argument errors first
+    assert call(0, 1, rows + 1) == fa.FA_ERR_INVALID_ARG
+    assert call(1, 1, rows + 1) == fa.FA_ERR_WORKSPACE
+    assert call(4, 8, rows // 32 + 1) == fa.FA_ERR_WORKSPACE
+
+
+# ---- the Python binding checks every tensor before taking its pointer ----
+
+def _host(shape, dtype="bf16"):
+    import torch
+    dt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[dtype]
+    return torch.zeros(shape, dtype=dt)
+
+
+def _fwd_args(B=2, H=3, Nq=40, Nk=56, D=64):
+    return dict(q=_host((B, H, Nq, D)), k=_host((B, H, Nk, D)), v=_host((B, H, Nk, D)),
+                o=_host((B, H, Nq, D)), lse=_host((B, H, Nq), "f32"))
+
+
+def _expect_invalid(fn, match, **kw):
+    with pytest.raises(fa.FaError, match=match) as e:
+        fn(**kw)
+    assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,bad,match", [
+    ("o", (2, 3, 39, 64), "o must have shape"),
+    ("o", (2, 3, 40, 128), "o must have shape"),
+    ("lse", (2, 3, 41), "lse must have shape"),
+    ("v", (2, 3, 55, 64), "v must have shape"),
+    ("k", (2, 4, 56, 64), "k must be"),
+    ("k", (2, 3, 56, 32), "k must be"),
+])
+def test_binding_rejects_misshaped_forward_tensors(L, name, bad, match):
+    kw = _fwd_args()
+    kw[name] = _host(bad, "f32" if name == "lse" else "bf16")
+    _expect_invalid(fa.fa_fwd, match, **kw)
+
+
+def test_binding_rejects_wrong_dtypes_layout_and_device(L):
+    kw = _fwd_args()
+    kw["v"] = _host((2, 3, 56, 64), "f16")
+    _expect_invalid(fa.fa_fwd, "v must be torch.bfloat16", **kw)
+    kw = _fwd_args()
+    kw["lse"] = _host((2, 3, 40), "bf16")
+    _expect_invalid(fa.fa_fwd, "lse must be torch.float32", **kw)
+    kw = _fwd_args()
+    kw["key_bias"] = _host((2, 55), "f32")
+    _expect_invalid(fa.fa_fwd, "key_bias must have shape", **kw)
+    kw = _fwd_args()
+    kw["key_bias"] = _host((2, 56), "bf16")
+    _expect_invalid(fa.fa_fwd, "key_bias must be torch.float32", **kw)
+    kw = _fwd_args()
+    kw["o"] = _host((2, 3, 64, 40)).transpose(2, 3)       # right shape, wrong layout
+    _expect_invalid(fa.fa_fwd, "contiguous", **kw)
+    kw = _fwd_args()                                       # everything right but on the host
+    _expect_invalid(fa.fa_fwd, "CUDA device", **kw)
+    kw = _fwd_args()
+    kw["q"] = _host((2, 3, 40, 64), "f32")
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_fwd(**kw)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("fn", ["fa_bwd", "fa_bwd_noalloc"])
+@pytest.mark.parametrize("name,bad", [("dq", (2, 3, 40, 32)), ("dk", (2, 3, 40, 64)),
+                                      ("dv", (2, 3, 57, 64)), ("dO", (2, 3, 40, 128)),
+                                      ("o", (1, 3, 40, 64))])
+def test_binding_rejects_misshaped_backward_tensors(L, fn, name, bad):
+    kw = _fwd_args()
+    kw.update(dO=_host((2, 3, 40, 64)), dq=_host((2, 3, 40, 64)), dk=_host((2, 3, 56, 64)),
+              dv=_host((2, 3, 56, 64)))
+    if fn == "fa_bwd":
+        kw["workspace"] = _host((fa.fa_bwd_workspace_bytes(2, 3, 40, 56, 64),), "f32")
+    kw[name] = _host(bad)
+    _expect_invalid(getattr(fa, fn), f"{name} must have shape", **kw)
+
+
+def test_binding_rejects_missing_outputs_and_host_workspace(L):
+    kw = _fwd_args()
+    kw.update(dO=_host((2, 3, 40, 64)), dq=None, dk=_host((2, 3, 56, 64)),
+              dv=_host((2, 3, 56, 64)), workspace=_host((4096,), "f32"))
+    _expect_invalid(fa.fa_bwd, "dq is required", **kw)
+    kw = _fwd_args()
+    kw["num_splits"] = 4
+    kw["workspace"] = _host((16,), "f32")
+    kw["o"] = _host((2, 3, 40, 32))
+    _expect_invalid(fa.fa_fwd_splitkv, "o must have shape", **kw)

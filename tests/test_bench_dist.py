@@ -61,7 +61,7 @@ def test_kernel_table_shares_and_flops():
 def test_sweep_overrides_name_and_batch():
     w = bench.workload_cfg(bench.parse_args(["--workload", "sweep", "--seq-len", "2048", "--causal", "0"]))
     assert (w["B"], w["Nq"], w["Nk"], w["causal"]) == (8, 2048, 2048, False)
-    assert w["name"] == "sweep-N2048-full"          # stored ncu traffic never matches it
+    assert w["name"] == "sweep-H16-N2048-full"      # stored ncu traffic never matches it
     w = bench.workload_cfg(bench.parse_args(["--workload", "sweep", "--seq-len", "32768"]))
     assert (w["B"], w["Nq"]) == (1, 32768)          # B = max(1, 16384 // N)
     with pytest.raises(SystemExit):
@@ -69,20 +69,29 @@ def test_sweep_overrides_name_and_batch():
 
 
 def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
-    # bench reports ncu DRAM bytes only while the CUDA sources hash to the
-    # revision the capture was taken from
+    # bench reports ncu DRAM bytes only while the kernel's own source file and
+    # the shared device headers hash to the revision the capture was taken from
     csrc = tmp_path / "exact_attention_112_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cu").write_text("// kernel v1\n")
+    (csrc / "fa_bwd.cu").write_text("// backward v1\n")
+    (csrc / "fa_fwd.cu").write_text("// forward v1\n")
+    (csrc / "fa_ptx.cuh").write_text("// primitives v1\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    rev = bench.kernel_rev()
+    rev = bench.kernel_rev("fa_bwd_dkdv_kernel")
     import json
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
         {"fa_bwd_dkdv_kernel:llama": {"kernel_rev": rev, "bytes_per_launch": 123}}))
     w = {"name": "llama"}
     assert bench.load_traffic("fa_bwd_dkdv_kernel", w) == 123
     assert bench.load_traffic("fa_fwd_kernel", w) is None
-    (csrc / "k.cu").write_text("// kernel v2\n")
-    assert bench.kernel_rev() != rev
+    assert bench.load_traffic("fa_bwd_dkdv_kernel", {"name": "bwd"}) is None
+    (csrc / "fa_fwd.cu").write_text("// forward v2\n")        # another kernel's file
+    (csrc / "fa_new.cu").write_text("// a new file\n")
+    assert bench.load_traffic("fa_bwd_dkdv_kernel", w) == 123
+    (csrc / "fa_ptx.cuh").write_text("// primitives v2\n")    # a shared header
+    assert bench.kernel_rev("fa_bwd_dkdv_kernel") != rev
+    assert bench.load_traffic("fa_bwd_dkdv_kernel", w) is None
+    (csrc / "fa_ptx.cuh").write_text("// primitives v1\n")
+    (csrc / "fa_bwd.cu").write_text("// backward v2\n")       # the kernel's own file
     assert bench.load_traffic("fa_bwd_dkdv_kernel", w) is None
