@@ -22,7 +22,8 @@ import threading
 __all__ = [
     "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
-    "lib", "library_path", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_noalloc",
+    "lib", "library_path", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes",
+    "fa_bwd_noalloc",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
             vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
             L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp]
             L.fa_fwd.restype = i
+            L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, vp, vp]
+            L.fa_fwd_fp8.restype = i
             L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
             L.fa_fwd_splitkv_workspace_bytes.restype = sz
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
@@ -129,7 +132,7 @@ def _bad(what, msg):
 
 
 def _validate(what, q, k, v, *, o=None, lse=None, dO=None, dq=None, dk=None, dv=None,
-              key_bias=None, workspace=None, outputs=()):
+              key_bias=None, workspace=None, outputs=(), fp8=False):
     """Check every tensor handed to the C ABI before its pointer is taken.
 
     The library sees only pointers and the sizes derived from ``q`` and ``k``,
@@ -138,12 +141,19 @@ def _validate(what, q, k, v, *, o=None, lse=None, dO=None, dq=None, dk=None, dv=
     [B,H,Nq,D] f16/bf16; k, v are [B,H,Nk,D] of q's dtype; o, dO, dq have q's
     shape and dtype; dk, dv have k's; lse is float32 [B,H,Nq]; key_bias is
     float32 [B,Nk]; every tensor (workspace included) is contiguous and on the
-    current CUDA device.  Returns (B, H, Nq, Nk, D, dtype code).
+    current CUDA device.  With ``fp8``, q, k, v are float8_e4m3fn and o is
+    bf16.  Returns (B, H, Nq, Nk, D, dtype code).
     """
     import torch
     if q is None or q.dim() != 4:
         _bad(what, "q must be a 4-D tensor [B, H, Nq, D]")
-    code = _dtype_code(q)
+    if fp8:
+        if q.dtype != torch.float8_e4m3fn:
+            raise FaError(FA_ERR_UNSUPPORTED, f"{what}: q must be torch.float8_e4m3fn, got {q.dtype}")
+        code, out_dt = None, torch.bfloat16
+    else:
+        code = _dtype_code(q)
+        out_dt = q.dtype
     B, H, Nq, D = q.shape
     if k is None or v is None:
         _bad(what, "k and v are required")
@@ -152,7 +162,7 @@ def _validate(what, q, k, v, *, o=None, lse=None, dO=None, dq=None, dk=None, dv=
     Nk = k.shape[2]
     want = {"q": (q, (B, H, Nq, D), q.dtype), "k": (k, (B, H, Nk, D), q.dtype),
             "v": (v, (B, H, Nk, D), q.dtype)}
-    for name, t, shape, dt in (("o", o, (B, H, Nq, D), q.dtype),
+    for name, t, shape, dt in (("o", o, (B, H, Nq, D), out_dt),
                                ("lse", lse, (B, H, Nq), torch.float32),
                                ("dO", dO, (B, H, Nq, D), q.dtype),
                                ("dq", dq, (B, H, Nq, D), q.dtype),
@@ -194,6 +204,20 @@ def fa_fwd(q, k, v, o, lse, causal=False, scale=None, key_bias=None, stream=None
                       int(bool(causal)), float(scale), code, _ptr(key_bias),
                       _stream_ptr(stream))
     _check(st, "fa_fwd")
+
+
+def fa_fwd_fp8(q, k, v, o, lse, causal=False, scale=None, q_descale=1.0, k_descale=1.0,
+               v_descale=1.0, key_bias=None, stream=None):
+    """FP8 forward: q, k, v float8_e4m3fn [B,H,N,128] standing for
+    q_descale*q, k_descale*k, v_descale*v; writes bf16 ``o`` and fp32 ``lse``."""
+    B, H, Nq, Nk, D, _ = _validate("fa_fwd_fp8", q, k, v, o=o, lse=lse, key_bias=key_bias,
+                                   outputs=("o", "lse"), fp8=True)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    st = lib().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
+                          int(bool(causal)), float(scale), float(q_descale), float(k_descale),
+                          float(v_descale), _ptr(key_bias), _stream_ptr(stream))
+    _check(st, "fa_fwd_fp8")
 
 
 def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits) -> int:

@@ -28,6 +28,7 @@ __device__ int g_fa_error_word;
 std::mutex g_mu;
 int *g_err_ptr[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int current_device(int *dev) {
@@ -36,21 +37,28 @@ int current_device(int *dev) {
     return FA_OK;
 }
 
-// Per-device set-up, done once: the error word's device address and the
-// compute capability.
-int device_setup(int dev, int **err_ptr) {
+// Per-device set-up, done once: the error word's device address, the
+// compute capability and the SM count (the persistent grid size).
+int device_setup(int dev, int **err_ptr, int *sm_count = nullptr) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_err_ptr[dev]) {
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FA_ERR_CUDA;
         g_cc_major[dev] = prop.major;
+        g_sm_count[dev] = prop.multiProcessorCount;
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_fa_error_word) != cudaSuccess) return FA_ERR_CUDA;
         g_err_ptr[dev] = static_cast<int *>(ptr);
     }
     if (g_cc_major[dev] != 10) return FA_ERR_UNSUPPORTED;
     *err_ptr = g_err_ptr[dev];
+    if (sm_count) *sm_count = g_sm_count[dev] > 0 ? g_sm_count[dev] : 1;
     return FA_OK;
+}
+
+// Persistent grid: one CTA per SM, or fewer when there are fewer units.
+int persistent_grid(long long units, int sm_count) {
+    return static_cast<int>(units < sm_count ? units : sm_count);
 }
 
 int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
@@ -67,19 +75,24 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
     return FA_OK;
 }
 
-// 3-D map over a [B*H, N, D] 16-bit tensor: box = 64 values x box_rows rows,
-// 128-byte swizzle (matches the MMA operand layout); rows past N read as 0
-// and are not written by stores.
-int make_map(CUtensorMap *m, const void *ptr, bool bf16, int D, int N, long long BH, int box_rows) {
+// 3-D map over a [B*H, N, D] tensor of 16-bit (or, with fp8, 8-bit) values:
+// box = one 128-byte row segment (64 or 128 values) x box_rows rows, 128-byte
+// swizzle (matches the MMA operand layout); rows past N read as 0 and are not
+// written by stores.
+int make_map(CUtensorMap *m, const void *ptr, bool bf16, int D, int N, long long BH, int box_rows,
+             bool fp8 = false) {
     PFN_cuTensorMapEncodeTiled_v12000 enc;
     int st = get_encoder(&enc);
     if (st != FA_OK) return st;
+    const cuuint64_t elem = fp8 ? 1 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem, static_cast<cuuint64_t>(N) * D * elem};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+    const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                       : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    CUresult r = enc(m, dt, 3,
                      const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -176,6 +189,35 @@ const char *fa_status_string(int status) {
     }
 }
 
+}  // extern "C"
+
+namespace {
+// Forward parameters shared by the forward entry points (one split).
+fa::FwdParams fwd_params(int B, int H, int Nq, int Nk, float scale, const float *key_bias, void *o,
+                         float *lse, int *err) {
+    fa::FwdParams p{};
+    p.B = B;
+    p.H = H;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.n_mblocks = (Nq + 255) / 256;
+    p.n_units = p.n_mblocks * B * H;
+    p.causal_off = Nk - Nq;
+    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    p.o_scale = 1.f;
+    p.bias = key_bias;
+    p.o = o;
+    p.lse = lse;
+    p.err = err;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.num_splits = 1;
+    p.tiles_per_split = 0;
+    return p;
+}
+}  // namespace
+
+extern "C" {
+
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int Nq,
            int Nk, int D, int causal, float scale, int dtype, const float *key_bias, void *stream) {
     int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
@@ -187,8 +229,8 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
         return FA_ERR_INVALID_ARG;
     int dev;
     if ((st = current_device(&dev)) != FA_OK) return st;
-    int *err = nullptr;
-    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    int *err = nullptr, sms = 1;
+    if ((st = device_setup(dev, &err, &sms)) != FA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
     const long long BH = static_cast<long long>(B) * H;
@@ -200,20 +242,46 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
     if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
     if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
-    if ((st = make_map(&tm.o, o, bf16, D, Nq, BH, 32)) != FA_OK) return st;
-    fa::FwdParams p;
-    p.B = B;
-    p.H = H;
-    p.Nq = Nq;
-    p.Nk = Nk;
-    p.n_mblocks = (Nq + 255) / 256;
-    p.causal_off = Nk - Nq;
-    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
-    p.bias = key_bias;
-    p.lse = lse;
-    p.err = err;
-    p.timeout_ns = kDefaultTimeoutNs;
-    cudaError_t e = fa::launch_fwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
+    fa::FwdParams p = fwd_params(B, H, Nq, Nk, scale, key_bias, o, lse, err);
+    cudaError_t e = fa::launch_fwd(tm, p, D, bf16 ? fa::kElemBF16 : fa::kElemF16, causal != 0,
+                                   key_bias != nullptr, persistent_grid(p.n_units, sms), s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+               int Nq, int Nk, int D, int causal, float scale, float q_descale, float k_descale,
+               float v_descale, const float *key_bias, void *stream) {
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, FA_BF16);
+    if (st != FA_OK) return st;
+    if (D != 128) return FA_ERR_UNSUPPORTED;
+    for (float d : {q_descale, k_descale, v_descale})
+        if (!std::isfinite(d) || !(d > 0.f)) return FA_ERR_INVALID_ARG;
+    const double qk = static_cast<double>(scale) * q_descale * k_descale;
+    if (!std::isfinite(qk) || qk <= 0.0 || qk > 3.0e38) return FA_ERR_INVALID_ARG;
+    if (Nq == 0) return FA_OK;
+    if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (key_bias && !aligned16(key_bias)))
+        return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr, sms = 1;
+    if ((st = device_setup(dev, &err, &sms)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long BH = static_cast<long long>(B) * H;
+    if (Nk == 0) {
+        return fa::launch_fwd_empty(o, lse, static_cast<size_t>(BH) * Nq, D, true, s) == cudaSuccess
+                   ? FA_OK : FA_ERR_CUDA;
+    }
+    fa::FwdTensorMaps tm;
+    if ((st = make_map(&tm.q, q, false, D, Nq, BH, 128, true)) != FA_OK) return st;
+    if ((st = make_map(&tm.k, k, false, D, Nk, BH, 128, true)) != FA_OK) return st;
+    if ((st = make_map(&tm.v, v, false, D, Nk, BH, 128, true)) != FA_OK) return st;
+    fa::FwdParams p = fwd_params(B, H, Nq, Nk, scale, key_bias, o, lse, err);
+    p.qk_scale_log2 = static_cast<float>(qk * 1.4426950408889634074);
+    p.o_scale = v_descale;
+    cudaError_t e = fa::launch_fwd(tm, p, D, fa::kElemE4M3, causal != 0, key_bias != nullptr,
+                                   persistent_grid(p.n_units, sms), s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -244,8 +312,8 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
     if (units > INT32_MAX) return FA_ERR_INVALID_ARG;
     int dev;
     if ((st = current_device(&dev)) != FA_OK) return st;
-    int *err = nullptr;
-    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    int *err = nullptr, sms = 1;
+    if ((st = device_setup(dev, &err, &sms)) != FA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == FA_BF16;
     const long long BH = static_cast<long long>(B) * H;
@@ -253,27 +321,17 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
     if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
     if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
     if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
-    if ((st = make_map(&tm.o, o, bf16, D, Nq, BH, 32)) != FA_OK) return st;
     const size_t rows = static_cast<size_t>(BH) * Nq * num_splits;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    fa::FwdParams p;
-    p.B = B;
-    p.H = H;
-    p.Nq = Nq;
-    p.Nk = Nk;
-    p.n_mblocks = (Nq + 255) / 256;
-    p.causal_off = Nk - Nq;
-    p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
-    p.bias = key_bias;
-    p.lse = lse;
-    p.err = err;
-    p.timeout_ns = kDefaultTimeoutNs;
+    fa::FwdParams p = fwd_params(B, H, Nq, Nk, scale, key_bias, o, lse, err);
     const int tiles = (Nk + 127) / 128;
     p.num_splits = num_splits;
     p.tiles_per_split = (tiles + num_splits - 1) / num_splits;
+    p.n_units = static_cast<int>(units);
     p.o_part = static_cast<float *>(workspace);
     p.lse_part = reinterpret_cast<float *>(static_cast<char *>(workspace) + up(rows * D * sizeof(float)));
-    cudaError_t e = fa::launch_fwd_split(tm, p, D, bf16, causal != 0, key_bias != nullptr, o, s);
+    cudaError_t e = fa::launch_fwd_split(tm, p, D, bf16, causal != 0, key_bias != nullptr,
+                                         persistent_grid(units, sms), s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -9,24 +9,33 @@
 // (m, l, o) update of "Online softmax: divide once, at the end"; O = o / l is
 // formed once per row after the last tile.
 //
-// B200 mapping (one CTA = one work unit of 256 query rows = two 128-row tiles
-// Q0, Q1 of one (batch, head)):
-//   * TMA streams Q once and K_j / V_j through a 2-stage shared-memory ring,
-//     handing each stage over with an mbarrier (expect_tx / complete_tx).
+// B200 mapping.  A work unit is 256 query rows (two 128-row tensor-core tiles
+// Q0, Q1) of one (batch, head), optionally restricted to one range of key
+// tiles (split-KV).  The kernel is persistent: one CTA per SM takes the units
+// in a fixed order (heaviest first -- the causal units that see the most key
+// tiles -- dealt out in a snake over the CTAs, which balances the causal
+// triangle as well as a greedy longest-first schedule), so tensor memory,
+// barriers and the pipeline are set up once per SM and the next unit's Q load
+// and first S products overlap the current unit's epilogue.
+//   * TMA streams Q (two tiles per unit, each released as soon as its last S
+//     product has read it; the next unit's Q is prefetched into L2 when the
+//     current unit starts) and K_j / V_j through a 2-stage shared-memory
+//     ring that runs on across unit boundaries, each stage handed over by an
+//     mbarrier (expect_tx / complete_tx).
 //   * The MMA warp issues tcgen05.mma from one elected lane while the whole
 //     warp runs the loop (warp-uniform descriptors and counters): S_i =
 //     Q_i K_j^T (both operands from shared memory, fp32 accumulator in tensor
 //     memory) and O_i += P_i V_j (P_i read from tensor memory, V_j from shared
-//     memory).
+//     memory).  16-bit inputs use kind::f16 (K = 16 per instruction); E4M3
+//     inputs use kind::f8f6f4 (K = 32) with P rounded to E4M3.
 //   * Two softmax warpgroups (one per Q tile, one thread per query row) read
 //     S_i from tensor memory, apply scale and mask in the base-2 domain
 //     (qk_scale = scale * log2(e), the constant derived in "Mastering
 //     FlashAttention: The Algebraic Foundation"), update the row max and sum in
-//     registers, write P_i back into the same tensor-memory columns as 16-bit
-//     values and signal the MMA warp.  While one warpgroup works on S_0 the
-//     tensor core computes S_1, and vice versa.  Three exponentials in four
-//     run on the MUFU unit, the fourth on the FMA pipe (exp2_fma2), so that
-//     the exponentials do not co-limit the loop with the tensor core.
+//     registers and write P_i back over the S_i columns in two halves of 64
+//     keys, each with its own barrier, so the first half of P_i V_j runs while
+//     the second half is still being exponentiated.  Three exponentials in
+//     four run on the MUFU unit, the fourth on the FMA pipe (exp2_fma2).
 //   * Lazy rescale: the reference maximum m_ref of a row only moves when a new
 //     tile's maximum exceeds it by more than kTau (log2 units); only then are
 //     l and the O accumulator multiplied by alpha = 2^(m_ref_old - m_ref_new).
@@ -34,14 +43,19 @@
 //     = e^(s - m_new): l, o and the final LSE all use the same m_ref.
 //   * Causal: key tiles entirely above the diagonal are never loaded or
 //     multiplied; tiles crossing it are masked per element.
+//   * Epilogue: each softmax thread divides its O row by l and stores it
+//     straight from registers (so the Q buffer is free for the next unit).
+//
+// MMA issue order (one in-order tensor pipe): per key tile t of a unit
+//     PV_0(t) [half 0, half 1], S_0(t+1), PV_1(t) [half 0, half 1], S_1(t+1)
+// and at a unit boundary PV_0(t), PV_1(t), S_0(next), S_1(next).
 //
 // Tensor memory (512 columns x 128 lanes of 32 bits; lane = query row):
-//   cols [0,128)        S_0 (fp32), later P_0 (16-bit pairs) in cols [0,64)
+//   cols [0,128)        S_0 (fp32), then P_0 over its first 64 (16-bit) or 32 (E4M3) columns
 //   cols [128,256)      S_1 / P_1
 //   cols [256,256+D)    O_0 accumulator (fp32)
 //   cols [256+D,256+2D) O_1 accumulator
-// Shared memory: Q_0, Q_1 (reused as O staging for the TMA store), K ring x2,
-// V ring x2, mbarriers.
+// Shared memory: Q_0, Q_1, K ring x2, V ring x2, mbarriers.
 //
 // Warp roles (12 warps): 0-3 softmax of Q_0, 4-7 softmax of Q_1, 8 TMA
 // producer, 9 MMA issuer (also allocates tensor memory), 10-11 idle (they
@@ -49,6 +63,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -77,34 +92,46 @@ constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
 constexpr int kEmuEvery = 4;        // one pair of exponentials in kEmuEvery on the FMA pipe
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+template <int D, int ELEM>
 struct FwdLayout {
-    static constexpr int kTileBytes = kBM * D * 2;       // one 128-row 16-bit tile
-    static constexpr int kChunkBytes = kBM * 128;        // 128 rows x 64 values
-    static constexpr int kQ = 0;                         // 2 tiles
-    static constexpr int kK = kQ + 2 * kTileBytes;       // kStages tiles
-    static constexpr int kV = kK + kStages * kTileBytes; // kStages tiles
+    static constexpr int kElemBytes = ELEM == kElemE4M3 ? 1 : 2;
+    static constexpr int kRowBytes = D * kElemBytes;      // one Q/K/V row
+    static constexpr int kChunkElems = 128 / kElemBytes;  // values per 128-byte swizzle row
+    static constexpr int kChunks = kRowBytes / 128;       // 128-byte column blocks per row
+    static constexpr int kTileBytes = kBM * kRowBytes;    // one 128-row tile
+    static constexpr int kChunkBytes = kBM * 128;         // 128 rows x 128 bytes
+    static constexpr int kKSteps = kRowBytes / 32;        // MMA K-steps of S (32 bytes each)
+    static constexpr int kPvKeys = 32 / kElemBytes;       // keys per P.V instruction
+    static constexpr int kPvSteps = kBN / kPvKeys;        // P.V instructions per tile
+    static constexpr int kPCols = kBN * kElemBytes / 4;   // tensor-memory columns of P
+    static constexpr int kQ = 0;                          // 2 tiles
+    static constexpr int kK = kQ + 2 * kTileBytes;        // kStages tiles
+    static constexpr int kV = kK + kStages * kTileBytes;  // kStages tiles
     static constexpr int kBar = kV + kStages * kTileBytes;
     // barrier indices
-    static constexpr int kQFull = 0;
-    static constexpr int kKFull = 1;     // +stage
-    static constexpr int kKEmpty = 3;    // +stage
-    static constexpr int kVFull = 5;     // +stage
-    static constexpr int kVEmpty = 7;    // +stage
-    static constexpr int kSFull = 9;     // +tile
-    static constexpr int kPFull = 11;    // +tile
-    static constexpr int kOFull = 13;    // +tile
-    static constexpr int kDrain = 15;
-    static constexpr int kNumBars = 16;
+    static constexpr int kQFull = 0;     // +tile
+    static constexpr int kQEmpty = 2;    // +tile
+    static constexpr int kKFull = 4;     // +stage
+    static constexpr int kKEmpty = 6;    // +stage
+    static constexpr int kVFull = 8;     // +stage
+    static constexpr int kVEmpty = 10;   // +stage
+    static constexpr int kSFull = 12;    // +tile
+    static constexpr int kPHalf = 14;    // +2*tile+half
+    static constexpr int kOFull = 18;    // +tile
+    static constexpr int kDrain = 20;
+    static constexpr int kNumBars = 21;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;       // room to align the base
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+    static_assert(kChunks >= 1 && kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle rows");
+    static_assert(kAlloc <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
+// Two fp32 values -> one 32-bit word of two 16-bit values (lo in the low half).
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     if constexpr (BF16) {
@@ -116,12 +143,74 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false>
+// Four fp32 values -> one 32-bit word of four E4M3 values (a in the low byte),
+// round to nearest even, saturating at the largest finite E4M3 value.
+__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+}
+
+// One work unit: rows [m0, m0 + 256) of head bh, key tiles
+// [kv_first, kv_first + n_kv) (n_kv == 0: the rows see no key).
+struct Unit {
+    int bh, m0, kv_first, n_kv, split;
+};
+
+template <bool CAUSAL, bool SPLIT>
+__device__ __forceinline__ Unit unit_info(const FwdParams &p, int u) {
+    Unit w;
+    const int BH = p.B * p.H;
+    w.split = 0;
+    if (SPLIT) {
+        w.split = u % p.num_splits;
+        u /= p.num_splits;
+    }
+    // heaviest (last) query blocks first
+    const int mb = (p.n_mblocks - 1) - u / BH;
+    w.bh = u % BH;
+    w.m0 = mb * 2 * kBM;
+    const int n_kv_all = (p.Nk + kBN - 1) / kBN;
+    w.n_kv = n_kv_all;
+    if (CAUSAL) {
+        const int last_row = min(w.m0 + 2 * kBM - 1, p.Nq - 1);
+        const int lim = last_row + p.causal_off;
+        w.n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kBN + 1);
+    }
+    w.kv_first = 0;
+    if (SPLIT) {
+        w.kv_first = w.split * p.tiles_per_split;
+        w.n_kv = max(0, min(w.n_kv, w.kv_first + p.tiles_per_split) - w.kv_first);
+    }
+    return w;
+}
+
+// r-th unit of this CTA in the snake order, or -1 when it has no more.
+__device__ __forceinline__ int unit_at(const FwdParams &p, int r) {
+    const int G = gridDim.x;
+    const long long u = static_cast<long long>(r) * G + ((r & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : blockIdx.x);
+    return u < p.n_units ? static_cast<int>(u) : -1;
+}
+
+// Advance r to this CTA's next unit that has key tiles (the producer and the
+// MMA warp skip the others); false when none is left.
+template <bool CAUSAL, bool SPLIT>
+__device__ __forceinline__ bool next_work(const FwdParams &p, int &r, Unit &w) {
+    for (;; ++r) {
+        const int u = unit_at(p, r);
+        if (u < 0) return false;
+        w = unit_info<CAUSAL, SPLIT>(p, u);
+        if (w.n_kv > 0) return true;
+    }
+}
+
+template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-              const FwdParams p) {
-    using L = FwdLayout<D>;
+              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using L = FwdLayout<D, ELEM>;
+    constexpr bool kFp8 = ELEM == kElemE4M3;
+    constexpr bool kOutBF16 = ELEM != kElemF16;   // O storage type
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -132,51 +221,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work unit: heaviest (last) query blocks first so that the hardware
-    // block scheduler hands the long causal units out early.  With SPLIT, the
-    // unit also names one contiguous range of key tiles.
     const int BH = p.B * p.H;
-    int unit = blockIdx.x;
-    int split = 0;
-    if (SPLIT) {
-        split = unit % p.num_splits;
-        unit /= p.num_splits;
-    }
-    const int mb = (p.n_mblocks - 1) - unit / BH;
-    const int bh = unit % BH;
-    const int m0 = mb * 2 * kBM;
-    const int n_kv_all = (p.Nk + kBN - 1) / kBN;
-    int n_kv = n_kv_all;      // key tiles this block may see
-    if (CAUSAL) {
-        const int last_row = min(m0 + 2 * kBM - 1, p.Nq - 1);
-        const int lim = last_row + p.causal_off;
-        n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kBN + 1);
-    }
-    int kv_first = 0;         // first key tile of this unit
-    if (SPLIT) {
-        kv_first = split * p.tiles_per_split;
-        n_kv = max(0, min(n_kv, kv_first + p.tiles_per_split) - kv_first);
-    }
 
-    // ---- set-up
+    // ---- set-up (once per CTA)
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        mbar_init(bar(L::kQFull), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(L::kQFull + i), 1);
+            mbar_init(bar(L::kQEmpty + i), 1);
+            mbar_init(bar(L::kSFull + i), 1);
+            mbar_init(bar(L::kPHalf + 2 * i), 4 * 32);
+            mbar_init(bar(L::kPHalf + 2 * i + 1), 4 * 32);
+            mbar_init(bar(L::kOFull + i), 1);
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(L::kKFull + s), 1);
             mbar_init(bar(L::kKEmpty + s), 1);
             mbar_init(bar(L::kVFull + s), 1);
             mbar_init(bar(L::kVEmpty + s), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bar(L::kSFull + i), 1);
-            mbar_init(bar(L::kPFull + i), 4 * 32);
-            mbar_init(bar(L::kOFull + i), 1);
         }
         mbar_init(bar(L::kDrain), 1);
         fence_mbar_init();
@@ -185,7 +251,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        prefetch_tmap(&tm_o);
     }
     tc_fence_before();
     __syncthreads();
@@ -200,28 +265,54 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp >= 8) regs_release<kRegsOther>();
     if (warp == kProducerWarp) {
         // ===================== TMA producer =====================
-        if (lane == 0 && n_kv > 0) {
-            int issued = 0;
+        if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTileBytes);
-            for (int i = 0; i < 2; ++i)
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &tm_q,
-                                bar(L::kQFull), c * 64, m0 + i * kBM, bh);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!mbar_wait(bar(L::kKEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
-                mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(sbase + L::kK + s * L::kTileBytes + c * L::kChunkBytes, &tm_k,
-                                bar(L::kKFull + s), c * 64, (kv_first + j) * kBN, bh);
-                if (!mbar_wait(bar(L::kVEmpty + s), ph ^ 1, wctx)) { ok = false; issued = 2 * j + 1; break; }
-                mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTileBytes);
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(sbase + L::kV + s * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                bar(L::kVFull + s), c * 64, (kv_first + j) * kBN, bh);
-                issued = 2 * j + 2;
+            int t = 0;          // key tiles loaded so far (ring position)
+            int uc = 0;         // units with key tiles started so far
+            int kv_half = 0;    // K and V loads issued (2 per key tile)
+            int q_issued = 0;   // Q tiles issued for the current unit
+            int r = 0;
+            Unit w;
+            while (ok && next_work<CAUSAL, SPLIT>(p, r, w)) {
+                // Q_i of this unit, once the previous unit's last S_i has read Q_i
+                q_issued = 0;
+                for (int i = 0; i < 2 && ok; ++i) {
+                    if (uc > 0 && !mbar_wait(bar(L::kQEmpty + i), (uc - 1) & 1, wctx)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar(L::kQFull + i), L::kTileBytes);
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_3d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &tm_q,
+                                    bar(L::kQFull + i), c * L::kChunkElems, w.m0 + i * kBM, w.bh);
+                    q_issued = i + 1;
+                }
+                if (!ok) break;
+                {   // warm L2 with the next unit's Q tiles
+                    int r2 = r + 1;
+                    Unit nx;
+                    if (next_work<CAUSAL, SPLIT>(p, r2, nx))
+                        for (int i = 0; i < 2; ++i)
+                            for (int c = 0; c < L::kChunks; ++c)
+                                tma_prefetch_l2_3d(&tm_q, c * L::kChunkElems, nx.m0 + i * kBM, nx.bh);
+                }
+                for (int j = 0; j < w.n_kv; ++j, ++t) {
+                    const int s = t & 1;
+                    const uint32_t ph = (t >> 1) & 1;
+                    const int row = (w.kv_first + j) * kBN;
+                    if (!mbar_wait(bar(L::kKEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_3d(sbase + L::kK + s * L::kTileBytes + c * L::kChunkBytes, &tm_k,
+                                    bar(L::kKFull + s), c * L::kChunkElems, row, w.bh);
+                    ++kv_half;
+                    if (!mbar_wait(bar(L::kVEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTileBytes);
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_3d(sbase + L::kV + s * L::kTileBytes + c * L::kChunkBytes, &tm_v,
+                                    bar(L::kVFull + s), c * L::kChunkElems, row, w.bh);
+                    ++kv_half;
+                }
+                if (!ok) break;
+                ++uc;
+                ++r;
             }
             if (!ok) {
                 // Give the copies already in flight a bounded chance to land
@@ -229,81 +320,137 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 WaitCtx drain{wctx.timeout_ns, wctx.err, nullptr};
                 volatile int zero = 0;
                 drain.abort_flag = &zero;
-                mbar_wait(bar(L::kQFull), 0, drain);
-                for (int t = (issued > 4 ? issued - 4 : 0); t < issued; ++t) {
-                    const int j = t >> 1;
-                    const int s = j & 1;
-                    const uint32_t ph = (j >> 1) & 1;
-                    mbar_wait(bar(((t & 1) ? L::kVFull : L::kKFull) + s), ph, drain);
+                for (int i = 0; i < q_issued; ++i) mbar_wait(bar(L::kQFull + i), uc & 1, drain);
+                for (int h = (kv_half > 4 ? kv_half - 4 : 0); h < kv_half; ++h) {
+                    const int tt = h >> 1;
+                    mbar_wait(bar(((h & 1) ? L::kVFull : L::kKFull) + (tt & 1)), (tt >> 1) & 1, drain);
                 }
             }
         }
         named_bar_sync(1, kThreads);
     } else if (warp == kMmaWarp) {
         // ============ MMA issuer (whole warp; one elected lane issues) ============
-        if (n_kv > 0) {
-            constexpr uint32_t idesc_qk = idesc_f16_f32acc(BF16, kBM, kBN, false, false);
-            constexpr uint32_t idesc_pv = idesc_f16_f32acc(BF16, kBM, D, false, true);
-            // S_i = Q_i K^T, then commit to `done` (and to `done2` if not 0)
-            auto issue_s = [&](int i, int stage, uint32_t done, uint32_t done2) {
+        int r = 0;
+        Unit w;
+        const bool have = next_work<CAUSAL, SPLIT>(p, r, w);
+        if (have) {
+            constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32acc(kBM, kBN, false, false)
+                                               : idesc_f16_f32acc(ELEM == kElemBF16, kBM, kBN, false, false);
+            constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32acc(kBM, D, false, true)
+                                               : idesc_f16_f32acc(ELEM == kElemBF16, kBM, D, false, true);
+            // S_i = Q_i K^T into the S_i columns; commits s_full(i), then
+            // k_empty(stage) after S_1, then q_empty(i) after a unit's last S_i
+            auto issue_s = [&](int i, int stage, bool release_k, bool release_q) {
                 const uint64_t dq = smem_desc_sw128(sbase + L::kQ + i * L::kTileBytes, 16, 1024);
                 const uint64_t dk = smem_desc_sw128(sbase + L::kK + stage * L::kTileBytes, 16, 1024);
                 const uint32_t d = tmem + (i ? L::kColS1 : L::kColS0);
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < L::kKSteps; ++kk) {
                         const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-                        umma_f16_ss(d, dq + off, dk + off, idesc_qk, kk > 0);
+                        if constexpr (kFp8)
+                            umma_f8_ss(d, dq + off, dk + off, idesc_qk, kk > 0);
+                        else
+                            umma_f16_ss(d, dq + off, dk + off, idesc_qk, kk > 0);
                     }
-                    umma_commit(done);
-                    if (done2) umma_commit(done2);
+                    umma_commit(bar(L::kSFull + i));
+                    if (release_k) umma_commit(bar(L::kKEmpty + stage));
+                    if (release_q) umma_commit(bar(L::kQEmpty + i));
                 }
                 __syncwarp();
             };
-            // O_i += P_i V (A: P_i over the S_i columns), then commit to `done` if not 0
-            auto issue_pv = [&](int i, int stage, bool acc, uint32_t done) {
+            // O_i += P_i V (A: P_i over the S_i columns), K-steps [k0, k1)
+            auto issue_pv = [&](int i, int stage, bool acc, int k0, int k1) {
                 const uint64_t dv = smem_desc_sw128(sbase + L::kV + stage * L::kTileBytes, L::kChunkBytes, 1024);
                 const uint32_t pa = tmem + (i ? L::kColS1 : L::kColS0);
                 const uint32_t d = tmem + (i ? L::kColO1 : L::kColO0);
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        umma_f16_ts(d, pa + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv,
-                                    (acc || kk > 0) ? 1u : 0u);
-                    if (done) umma_commit(done);
+                    for (int kk = 0; kk < L::kPvSteps; ++kk) {
+                        if (kk < k0 || kk >= k1) continue;
+                        const uint64_t b = dv + ((kk * L::kPvKeys * 128) >> 4);
+                        if constexpr (kFp8)
+                            umma_f8_ts(d, pa + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                        else
+                            umma_f16_ts(d, pa + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    }
                 }
                 __syncwarp();
             };
-            bool ok = mbar_wait_warp(bar(L::kQFull), 0, wctx) && mbar_wait_warp(bar(L::kKFull + 0), 0, wctx);
+            auto commit = [&](uint32_t b) {
+                if (elect_one()) umma_commit(b);
+                __syncwarp();
+            };
+            constexpr int kHalf = L::kPvSteps / 2;
+            int t = 0;      // key tiles issued so far (ring position, S/P barrier phases)
+            int uc = 0;     // units done so far (Q and O barrier phases)
+            bool ok = mbar_wait_warp(bar(L::kQFull + 0), 0, wctx) && mbar_wait_warp(bar(L::kKFull + 0), 0, wctx);
             if (ok) {
                 tc_fence_after();
-                issue_s(0, 0, bar(L::kSFull + 0), 0u);
-                issue_s(1, 0, bar(L::kSFull + 1), n_kv > 2 ? bar(L::kKEmpty + 0) : 0u);
+                issue_s(0, 0, false, w.n_kv == 1);
+                ok = mbar_wait_warp(bar(L::kQFull + 1), 0, wctx);
             }
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                const bool more = j + 1 < n_kv;
-                const int s2 = (j + 1) & 1;
-                const uint32_t ph2 = ((j + 1) >> 1) & 1;
-                if (!mbar_wait_warp(bar(L::kVFull + s), ph, wctx)) { ok = false; break; }
-                if (!mbar_wait_warp(bar(L::kPFull + 0), j & 1, wctx)) { ok = false; break; }
+            if (ok) {
                 tc_fence_after();
-                issue_pv(0, s, j > 0, more ? 0u : bar(L::kOFull + 0));
-                if (more) {
-                    if (!mbar_wait_warp(bar(L::kKFull + s2), ph2, wctx)) { ok = false; break; }
+                issue_s(1, 0, true, w.n_kv == 1);
+            }
+            while (ok) {
+                for (int j = 0; j < w.n_kv && ok; ++j, ++t) {
+                    const int s = t & 1;
+                    const uint32_t ph = (t >> 1) & 1;
+                    const bool last = j + 1 == w.n_kv;
+                    int r2 = r + 1;
+                    Unit nx = w;
+                    const bool has_next = !last || next_work<CAUSAL, SPLIT>(p, r2, nx);
+                    const int s1 = (t + 1) & 1;
+                    const uint32_t ph1 = ((t + 1) >> 1) & 1;
+                    const uint32_t pp = t & 1;
+                    if (!mbar_wait_warp(bar(L::kVFull + s), ph, wctx)) { ok = false; break; }
+                    // ---- P_0 V(t), half by half
+                    if (!mbar_wait_warp(bar(L::kPHalf + 0), pp, wctx)) { ok = false; break; }
                     tc_fence_after();
-                    issue_s(0, s2, bar(L::kSFull + 0), 0u);
+                    issue_pv(0, s, j > 0, 0, kHalf);
+                    if (!mbar_wait_warp(bar(L::kPHalf + 1), pp, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(0, s, j > 0, kHalf, L::kPvSteps);
+                    if (last) commit(bar(L::kOFull + 0));
+                    // ---- S_0(t+1) inside the unit
+                    if (!last) {
+                        if (!mbar_wait_warp(bar(L::kKFull + s1), ph1, wctx)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_s(0, s1, false, j + 2 == w.n_kv);
+                    }
+                    // ---- P_1 V(t)
+                    if (!mbar_wait_warp(bar(L::kPHalf + 2), pp, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, s, j > 0, 0, kHalf);
+                    if (!mbar_wait_warp(bar(L::kPHalf + 3), pp, wctx)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(1, s, j > 0, kHalf, L::kPvSteps);
+                    commit(bar(L::kVEmpty + s));
+                    if (last) commit(bar(L::kOFull + 1));
+                    // ---- S_1(t+1), or both S products of the next unit's first tile
+                    if (has_next) {
+                        if (last) {
+                            if (!mbar_wait_warp(bar(L::kQFull + 0), (uc + 1) & 1, wctx) ||
+                                !mbar_wait_warp(bar(L::kKFull + s1), ph1, wctx)) { ok = false; break; }
+                            tc_fence_after();
+                            issue_s(0, s1, false, nx.n_kv == 1);
+                            if (!mbar_wait_warp(bar(L::kQFull + 1), (uc + 1) & 1, wctx)) { ok = false; break; }
+                            tc_fence_after();
+                            issue_s(1, s1, true, nx.n_kv == 1);
+                        } else {
+                            issue_s(1, s1, true, j + 2 == w.n_kv);
+                        }
+                    }
                 }
-                if (!mbar_wait_warp(bar(L::kPFull + 1), j & 1, wctx)) { ok = false; break; }
-                tc_fence_after();
-                issue_pv(1, s, j > 0, j + 2 < n_kv ? bar(L::kVEmpty + s) : 0u);
-                if (more)
-                    issue_s(1, s2, bar(L::kSFull + 1), j + 3 < n_kv ? bar(L::kKEmpty + s2) : 0u);
-                else if (elect_one())
-                    umma_commit(bar(L::kOFull + 1));
-                __syncwarp();
+                if (!ok) break;
+                ++uc;
+                ++r;
+                if (!next_work<CAUSAL, SPLIT>(p, r, w)) break;
             }
+        }
+        if (have) {
             // Every issued MMA must finish before tensor memory is released.
             if (elect_one()) umma_commit(bar(L::kDrain));
             __syncwarp();
@@ -322,94 +469,99 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int i = warp >> 2;            // which Q tile
         const int wq = warp & 3;            // lane quarter of tensor memory
         const int row = wq * 32 + lane;     // row within the tile (= TMEM lane)
-        const int qrow = m0 + i * kBM + row;
         const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t tS = tl + (i ? L::kColS1 : L::kColS0);
         const uint32_t tO = tl + (i ? L::kColO1 : L::kColO0);
         const float qk = p.qk_scale_log2;
-        // last key index this row may see
-        const int lim = CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1;
-        const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(bh / p.H) * p.Nk : nullptr;
-
-        float m_ref = neg_inf();   // log2 units
-        float l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const int kv0 = (kv_first + j) * kBN;
-            {
-                const bool got = mbar_wait(bar(L::kSFull + i), j & 1, wctx);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            }
-            tc_fence_after();
-            uint32_t sr[128];
-            tmem_ld32dp_x128_wait(tS, sr);
-            float x[128];
-            if constexpr (HAS_BIAS) {
-                // x = s * qk_scale + bias * log2(e); every lane reads the same
-                // addresses, so each load is one broadcast transaction.
-                constexpr float kLog2e = 1.4426950408889634f;
-                const float *bt = bias_b + kv0;
-                if (kv0 + kBN <= p.Nk && (reinterpret_cast<uintptr_t>(bt) & 15) == 0) {
-                    const float4 *b4 = reinterpret_cast<const float4 *>(bt);
+        int t = 0;      // key tiles seen so far (S/P barrier phases)
+        int uc = 0;     // units with key tiles done so far (O barrier phase)
+        for (int r = 0; ok; ++r) {
+            const int u = unit_at(p, r);
+            if (u < 0) break;
+            const Unit w = unit_info<CAUSAL, SPLIT>(p, u);
+            const int qrow = w.m0 + i * kBM + row;
+            // last key index this row may see
+            const int lim = CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1;
+            const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(w.bh / p.H) * p.Nk : nullptr;
+            float m_ref = neg_inf();   // log2 units
+            float l = 0.f;
+            for (int j = 0; j < w.n_kv; ++j, ++t) {
+                const int kv0 = (w.kv_first + j) * kBN;
+                {
+                    const bool got = mbar_wait(bar(L::kSFull + i), t & 1, wctx);
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                }
+                tc_fence_after();
+                uint32_t sr[128];
+                tmem_ld32dp_x128_wait(tS, sr);
+                float x[128];
+                if constexpr (HAS_BIAS) {
+                    // x = s * qk_scale + bias * log2(e); every lane reads the same
+                    // addresses, so each load is one broadcast transaction.
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    const float *bt = bias_b + kv0;
+                    if (kv0 + kBN <= p.Nk && (reinterpret_cast<uintptr_t>(bt) & 15) == 0) {
+                        const float4 *b4 = reinterpret_cast<const float4 *>(bt);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float4 bb = __ldg(b4 + c);
-                        x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, bb.x * kLog2e);
-                        x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, bb.y * kLog2e);
-                        x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, bb.z * kLog2e);
-                        x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, bb.w * kLog2e);
+                        for (int c = 0; c < 32; ++c) {
+                            const float4 bb = __ldg(b4 + c);
+                            x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, bb.x * kLog2e);
+                            x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, bb.y * kLog2e);
+                            x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, bb.z * kLog2e);
+                            x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, bb.w * kLog2e);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c) {
+                            const float bb = (kv0 + c < p.Nk) ? __ldg(bt + c) * kLog2e : 0.f;
+                            x[c] = fmaf(__uint_as_float(sr[c]), qk, bb);
+                        }
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const float bb = (kv0 + c < p.Nk) ? __ldg(bt + c) * kLog2e : 0.f;
-                        x[c] = fmaf(__uint_as_float(sr[c]), qk, bb);
-                    }
+                    for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
                 }
-            } else {
+                if (kv0 + kBN - 1 > lim) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-            }
-            if (kv0 + kBN - 1 > lim) {
+                    for (int c = 0; c < 128; ++c)
+                        if (kv0 + c > lim) x[c] = neg_inf();
+                }
+                float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (kv0 + c > lim) x[c] = neg_inf();
-            }
-            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
-#pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, x[c]);
-                mx1 = fmaxf(mx1, x[c + 1]);
-                mx2 = fmaxf(mx2, x[c + 2]);
-                mx3 = fmaxf(mx3, x[c + 3]);
-            }
-            float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            if constexpr (!HAS_BIAS) m_tile *= qk;   // qk > 0: max commutes with scaling
-            const bool need = m_tile > m_ref + kTau;
-            // warp-uniform: if any row of the warp moves its reference maximum,
-            // the warp rescales its O rows (after P is formed, below)
-            const bool rescale = __any_sync(0xffffffffu, need);
-            float alpha = 1.f;
-            if (rescale) {
-                const float m_new = need ? m_tile : m_ref;
-                alpha = (m_ref == neg_inf()) ? 0.f : ex2_approx(m_ref - m_new);
-                l *= alpha;
-                m_ref = m_new;
-            }
-            const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
-            // p = 2^(x - m), two columns per paired-fp32 instruction.  P goes
-            // back into the S columns in two halves (every S value is already
-            // in registers), which keeps the live registers low.  On tiles
-            // without masked scores, one pair in kEmuEvery goes through the
-            // FMA-pipe exponential instead of MUFU.
-            float2 lsum = make_float2(0.f, 0.f);
-            const float2 neg_m2 = make_float2(-m_use, -m_use);
-            const float2 qk2 = make_float2(qk, qk);
-            auto make_p = [&](auto emu_tag) {
-                constexpr bool kEmu = decltype(emu_tag)::value;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[32];
+                for (int c = 4; c < 128; c += 4) {
+                    mx0 = fmaxf(mx0, x[c]);
+                    mx1 = fmaxf(mx1, x[c + 1]);
+                    mx2 = fmaxf(mx2, x[c + 2]);
+                    mx3 = fmaxf(mx3, x[c + 3]);
+                }
+                float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                if constexpr (!HAS_BIAS) m_tile *= qk;   // qk > 0: max commutes with scaling
+                const bool need = m_tile > m_ref + kTau;
+                // warp-uniform: if any row of the warp moves its reference maximum,
+                // the warp rescales its O rows (before the first half of P is
+                // handed over, below)
+                const bool rescale = __any_sync(0xffffffffu, need);
+                float alpha = 1.f;
+                if (rescale) {
+                    const float m_new = need ? m_tile : m_ref;
+                    alpha = (m_ref == neg_inf()) ? 0.f : ex2_approx(m_ref - m_new);
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
+                // p = 2^(x - m), two columns per paired-fp32 instruction, in two
+                // halves of 64 keys; each half goes back over the S columns and
+                // is handed to the MMA warp on its own barrier.  On tiles without
+                // masked scores, one pair in kEmuEvery goes through the FMA-pipe
+                // exponential instead of MUFU.
+                float2 lsum = make_float2(0.f, 0.f);
+                const float2 neg_m2 = make_float2(-m_use, -m_use);
+                const float2 qk2 = make_float2(qk, qk);
+                const bool emu = __all_sync(0xffffffffu, !HAS_BIAS && kv0 + kBN - 1 <= lim);   // warp-uniform
+                auto half = [&](int h, auto emu_tag) {
+                    constexpr bool kEmu = decltype(emu_tag)::value;
+                    float pv[64];
 #pragma unroll
                     for (int c2 = 0; c2 < 32; ++c2) {
                         const int c = 64 * h + 2 * c2;
@@ -421,111 +573,112 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         else
                             pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                         lsum = __fadd2_rn(lsum, pp);
-                        pk[c2] = pack2<BF16>(pp.x, pp.y);
+                        pv[2 * c2] = pp.x;
+                        pv[2 * c2 + 1] = pp.y;
                     }
-                    tmem_st32dp_x32(tS + 32 * h, pk);
+                    if constexpr (kFp8) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack4_e4m3(pv[4 * e], pv[4 * e + 1], pv[4 * e + 2], pv[4 * e + 3]);
+                        tmem_st32dp_x16(tS + 16 * h, pk);
+                    } else {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pk[e] = pack2<ELEM == kElemBF16>(pv[2 * e], pv[2 * e + 1]);
+                        tmem_st32dp_x32(tS + 32 * h, pk);
+                    }
+                };
+                if (emu)
+                    half(0, std::true_type{});
+                else
+                    half(0, std::false_type{});
+                if (rescale && j > 0) {
+                    // O_i row *= alpha.  O is stable: the MMA that produced this
+                    // S tile was issued after the previous P.V and its commit
+                    // covers it; the next P.V waits for the arrive below.
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orr[32];
+                        tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32dp_x32(tO + cc * 32, orr);
+                    }
                 }
-            };
-            // warp-uniform choice: make_p holds warp-collective tensor-memory stores
-            if (__all_sync(0xffffffffu, !HAS_BIAS && kv0 + kBN - 1 <= lim))
-                make_p(std::true_type{});
-            else
-                make_p(std::false_type{});
-            const float l0 = lsum.x, l1 = lsum.y;
-            l += l0 + l1;
-            if (rescale && j > 0) {
-                // O_i row *= alpha.  O is stable: the MMA that produced this S
-                // tile was issued after the previous P.V and its commit covers
-                // it; the next P.V waits for the arrive below.
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::kPHalf + 2 * i));
+                if (emu)
+                    half(1, std::true_type{});
+                else
+                    half(1, std::false_type{});
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::kPHalf + 2 * i + 1));
+                l += lsum.x + lsum.y;
+            }
+            if (!ok) break;
+
+            // ---- epilogue: O = o / l (times o_scale), LSE = (m_ref + log2 l) ln 2
+            if (w.n_kv > 0) {
+                const bool got = mbar_wait(bar(L::kOFull + i), uc & 1, wctx);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                ++uc;
+            }
+            const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
+            const float lse = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : neg_inf();
+            if (SPLIT) {
+                // partial result of this key range: O_s = o / l (fp32), LSE_s
+                const size_t prow = (static_cast<size_t>(w.split) * BH + w.bh) * p.Nq + qrow;
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t orr[32];
-                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+                    if (w.n_kv > 0) {
+                        tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32dp_x32(tO + cc * 32, orr);
+                        for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                    }
+                    if (qrow < p.Nq) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o_part + prow * D + cc * 32);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
+                                                 __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
+                    }
                 }
+                if (qrow < p.Nq) p.lse_part[prow] = lse;
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) +
+                                                       (static_cast<size_t>(w.bh) * p.Nq + qrow) * D);
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t orr[32];
+                    if (w.n_kv > 0) {
+                        tmem_ld32dp_x32_wait(tO + cc * 32, orr);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack2<kOutBF16>(__uint_as_float(orr[2 * e]) * inv_l,
+                                                __uint_as_float(orr[2 * e + 1]) * inv_l);
+                    if (qrow < p.Nq) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                    }
+                }
+                if (qrow < p.Nq) p.lse[static_cast<size_t>(w.bh) * p.Nq + qrow] = lse;
             }
-            tmem_wait_st();
+            // the next unit's first P.V may overwrite O_i only after these loads
             tc_fence_before();
-            mbar_arrive(bar(L::kPFull + i));
         }
-
-        // ---- epilogue: O = o / l, LSE = (m_ref + log2 l) ln 2
-        if (ok && n_kv > 0) {
-            const bool got = mbar_wait(bar(L::kOFull + i), 0, wctx);
-            ok = __all_sync(0xffffffffu, got);
-            tc_fence_after();
-        }
-        if (ok && SPLIT) {
-            // partial result of this key range: O_s = o / l (fp32), LSE_s
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            const size_t prow = (static_cast<size_t>(split) * BH + bh) * p.Nq + qrow;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t orr[32];
-                if (n_kv > 0) {
-                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
-                }
-                if (qrow < p.Nq) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + prow * D + cc * 32);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
-                                             __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
-                }
-            }
-            if (qrow < p.Nq)
-                p.lse_part[prow] = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : neg_inf();
-        } else if (ok) {
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            uint8_t *stage = smem + L::kQ + i * L::kTileBytes;   // Q_i is dead now
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t orr[32];
-                if (n_kv > 0) {
-                    tmem_ld32dp_x32_wait(tO + cc * 32, orr);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
-                                        __uint_as_float(orr[2 * e + 1]) * inv_l);
-                // 128-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)
-                const int chunk = (cc * 32) / 64;
-                const int k16_base = ((cc * 32) % 64) / 8;
-                uint8_t *rowp = stage + chunk * L::kChunkBytes + row * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int k16 = (k16_base + q4) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(rowp + k16 * 16) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-                }
-            }
-            if (qrow < p.Nq) {
-                const float lse = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : neg_inf();
-                p.lse[static_cast<size_t>(bh) * p.Nq + qrow] = lse;
-            }
-            // each warp stores its own 32 rows (box 64 x 32)
-            fence_proxy_async_smem();
-            __syncwarp();
-            const int row0 = m0 + i * kBM + wq * 32;
-            if (lane == 0 && row0 < p.Nq) {
-                for (int c = 0; c < D / 64; ++c)
-                    tma_store_3d(&tm_o, sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes + wq * 32 * 128,
-                                 c * 64, row0, bh);
-                tma_store_commit();
-                tma_store_wait_all();
-            }
-        }
-        tc_fence_before();
         named_bar_sync(1, kThreads);
     } else {
         named_bar_sync(1, kThreads);   // idle warps 10, 11
@@ -584,36 +737,35 @@ __global__ void fa_fwd_empty_kernel(T *o, float *lse, size_t n_rows, int D) {
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, cudaStream_t stream) {
-    using L = FwdLayout<D>;
-    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS>
+cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
+    using L = FwdLayout<D, ELEM>;
+    auto kern = fa_fwd_kernel<D, ELEM, CAUSAL, HAS_BIAS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H;
     prof_begin(stream, "fa_fwd_kernel");
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     return cudaGetLastError();
 }
 
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
-cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, void *o, cudaStream_t stream) {
-    using L = FwdLayout<D>;
-    auto kern = fa_fwd_kernel<D, BF16, CAUSAL, HAS_BIAS, true>;
+cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
+    constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
+    using L = FwdLayout<D, kElem>;
+    auto kern = fa_fwd_kernel<D, kElem, CAUSAL, HAS_BIAS, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.H * p.num_splits;
     prof_begin(stream, "fa_fwd_split_kernel");
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, tm.o, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
     const unsigned cgrid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
     prof_begin(stream, "fa_fwd_combine_kernel");
-    fa_fwd_combine_kernel<D, BF16><<<cgrid, 256, 0, stream>>>(p.o_part, p.lse_part, static_cast<uint16_t *>(o),
+    fa_fwd_combine_kernel<D, BF16><<<cgrid, 256, 0, stream>>>(p.o_part, p.lse_part, static_cast<uint16_t *>(p.o),
                                                                p.lse, rows, p.num_splits);
     prof_end(stream);
     note_launch();
@@ -621,35 +773,36 @@ cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, void *o,
 }
 
 template <int D, bool BF16>
-cudaError_t launch_split_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias, void *o,
+cudaError_t launch_split_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias, int grid,
                            cudaStream_t s) {
-    if (causal) return bias ? launch_split_t<D, BF16, true, true>(tm, p, o, s) : launch_split_t<D, BF16, true, false>(tm, p, o, s);
-    return bias ? launch_split_t<D, BF16, false, true>(tm, p, o, s) : launch_split_t<D, BF16, false, false>(tm, p, o, s);
+    if (causal) return bias ? launch_split_t<D, BF16, true, true>(tm, p, grid, s) : launch_split_t<D, BF16, true, false>(tm, p, grid, s);
+    return bias ? launch_split_t<D, BF16, false, true>(tm, p, grid, s) : launch_split_t<D, BF16, false, false>(tm, p, grid, s);
 }
 
-template <int D, bool BF16>
-cudaError_t launch_fwd_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias,
+template <int D, int ELEM>
+cudaError_t launch_fwd_d(const FwdTensorMaps &tm, const FwdParams &p, bool causal, bool bias, int grid,
                          cudaStream_t s) {
-    if (causal) return bias ? launch_fwd_t<D, BF16, true, true>(tm, p, s) : launch_fwd_t<D, BF16, true, false>(tm, p, s);
-    return bias ? launch_fwd_t<D, BF16, false, true>(tm, p, s) : launch_fwd_t<D, BF16, false, false>(tm, p, s);
+    if (causal) return bias ? launch_fwd_t<D, ELEM, true, true>(tm, p, grid, s) : launch_fwd_t<D, ELEM, true, false>(tm, p, grid, s);
+    return bias ? launch_fwd_t<D, ELEM, false, true>(tm, p, grid, s) : launch_fwd_t<D, ELEM, false, false>(tm, p, grid, s);
 }
 
 }  // namespace
 
-cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
-                       bool has_bias, cudaStream_t stream) {
-    if (D == 64) return bf16 ? launch_fwd_d<64, true>(tm, p, causal, has_bias, stream)
-                             : launch_fwd_d<64, false>(tm, p, causal, has_bias, stream);
-    return bf16 ? launch_fwd_d<128, true>(tm, p, causal, has_bias, stream)
-                : launch_fwd_d<128, false>(tm, p, causal, has_bias, stream);
+cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, int elem, bool causal,
+                       bool has_bias, int grid, cudaStream_t stream) {
+    if (elem == kElemE4M3) return launch_fwd_d<128, kElemE4M3>(tm, p, causal, has_bias, grid, stream);
+    if (D == 64) return elem == kElemBF16 ? launch_fwd_d<64, kElemBF16>(tm, p, causal, has_bias, grid, stream)
+                                          : launch_fwd_d<64, kElemF16>(tm, p, causal, has_bias, grid, stream);
+    return elem == kElemBF16 ? launch_fwd_d<128, kElemBF16>(tm, p, causal, has_bias, grid, stream)
+                             : launch_fwd_d<128, kElemF16>(tm, p, causal, has_bias, grid, stream);
 }
 
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
-                             bool has_bias, void *o, cudaStream_t stream) {
-    if (D == 64) return bf16 ? launch_split_d<64, true>(tm, p, causal, has_bias, o, stream)
-                             : launch_split_d<64, false>(tm, p, causal, has_bias, o, stream);
-    return bf16 ? launch_split_d<128, true>(tm, p, causal, has_bias, o, stream)
-                : launch_split_d<128, false>(tm, p, causal, has_bias, o, stream);
+                             bool has_bias, int grid, cudaStream_t stream) {
+    if (D == 64) return bf16 ? launch_split_d<64, true>(tm, p, causal, has_bias, grid, stream)
+                             : launch_split_d<64, false>(tm, p, causal, has_bias, grid, stream);
+    return bf16 ? launch_split_d<128, true>(tm, p, causal, has_bias, grid, stream)
+                : launch_split_d<128, false>(tm, p, causal, has_bias, grid, stream);
 }
 
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16, cudaStream_t stream) {

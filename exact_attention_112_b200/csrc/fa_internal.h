@@ -9,13 +9,19 @@
 
 namespace fa {
 
+// Storage types of Q, K, V (O is 16-bit: the input type, or bf16 for E4M3).
+enum ElemType : int { kElemF16 = 0, kElemBF16 = 1, kElemE4M3 = 2 };
+
 // Forward launch parameters (everything except the tensor maps).
 struct FwdParams {
     int B, H, Nq, Nk;
     int n_mblocks;                 // ceil(Nq / 256): work units per (b, h)
+    int n_units;                   // n_mblocks * B * H (* num_splits)
     int causal_off;                // Nk - Nq (bottom-right causal alignment)
-    float qk_scale_log2;           // scale * log2(e)
+    float qk_scale_log2;           // scale * log2(e) (E4M3: times the Q and K descales)
+    float o_scale;                 // multiplies O = o / l at the end (E4M3: the V descale)
     const float *bias;             // [B, Nk] or nullptr
+    void *o;                       // [B*H, Nq, D] 16-bit output
     float *lse;                    // [B*H, Nq]
     int *err;                      // device error word
     unsigned long long timeout_ns; // limit of every device-side wait
@@ -27,7 +33,7 @@ struct FwdParams {
 };
 
 struct FwdTensorMaps {
-    CUtensorMap q, k, v, o;
+    CUtensorMap q, k, v;
 };
 
 // Backward launch parameters.
@@ -59,10 +65,12 @@ void note_launch(unsigned n = 1);
 void prof_begin(cudaStream_t stream, const char *name);
 void prof_end(cudaStream_t stream);
 
-cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
-                       bool has_bias, cudaStream_t stream);
+// Persistent launches: `grid` CTAs (at most one per SM) take the p.n_units
+// work units in a fixed snake order.
+cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, int elem, bool causal,
+                       bool has_bias, int grid, cudaStream_t stream);
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
-                             bool has_bias, void *o, cudaStream_t stream);
+                             bool has_bias, int grid, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,
                              cudaStream_t stream);
 

@@ -29,7 +29,7 @@ import math
 import numpy as np
 import torch
 
-DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
+DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}
 
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384, 32768)
 
@@ -73,12 +73,14 @@ def _randn(shape, gen, std):
 
 def make_inputs(B, H, Nq, Nk, D, dtype="bf16", seed=0, qk_std=1.0,
                 v_dist="normal", bias_frac=0.0, with_dO=False, **_ignored):
-    """Draw Q, K, V (and dO) on the host, rounded to the 16-bit dtype.
+    """Draw Q, K, V (and dO) on the host, rounded to the storage dtype.
 
-    Returns a dict of CPU tensors: q [B,H,Nq,D], k/v [B,H,Nk,D] (16-bit),
-    optional do [B,H,Nq,D] (16-bit) and key_bias [B,Nk] float32 (or None).
-    The rounding (round-to-nearest-even, torch's cast) happens here, once, so
-    the oracle receives exactly the values the kernels read.
+    Returns a dict of CPU tensors: q [B,H,Nq,D], k/v [B,H,Nk,D] (16-bit, or
+    8-bit E4M3 for dtype "e4m3"), optional do [B,H,Nq,D] and key_bias [B,Nk]
+    float32 (or None).  The rounding (round-to-nearest-even, torch's cast)
+    happens here, once, so the oracle receives exactly the values the kernels
+    read.  E4M3 draws are far inside its range (|x| <= 448), so the cast never
+    saturates.
     """
     tdt = DTYPES[dtype]
     gen = torch.Generator(device="cpu").manual_seed(int(seed))

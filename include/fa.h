@@ -80,6 +80,26 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            int dtype, const float *key_bias, void *stream);
 
 /*
+ * Forward pass with 8-bit floating-point inputs, the low-precision tensor-core
+ * path the lastdictionary.com "FlashAttention" entry credits to
+ * FlashAttention-3 (definition paragraph: "exploited asynchrony and FP8").
+ *   q, k, v    [B,H,N,D] OCP FP8 E4M3 values (1 byte each, the finite-only
+ *              "e4m3fn" encoding); D must be 128.  The attention inputs are
+ *              q_descale * q, k_descale * k and v_descale * v (per-tensor
+ *              scale factors, finite and > 0; 1 for unscaled data).
+ *   o          [B,H,Nq,D] bf16;  lse [B,H,Nq] float32 as in fa_fwd().
+ * S = Q K^T runs on the tensor cores with E4M3 operands and an fp32
+ * accumulator; the probabilities P are rounded to E4M3 (round to nearest
+ * even) for the P V product, while the row sum l adds the unrounded fp32
+ * values.  Everything else (masking, causal alignment, empty rows, errors)
+ * is as in fa_fwd().  D != 128 returns FA_ERR_UNSUPPORTED.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+               int B, int H, int Nq, int Nk, int D, int causal, float scale,
+               float q_descale, float k_descale, float v_descale,
+               const float *key_bias, void *stream);
+
+/*
  * Split-KV forward, for few query rows and many keys (decoding): the keys are
  * cut into num_splits contiguous ranges of whole 128-key tiles, each range is
  * processed by its own CTAs into a partial (O_s, LSE_s) in fp32, and a second

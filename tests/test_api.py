@@ -255,3 +255,37 @@ def test_binding_rejects_missing_outputs_and_host_workspace(L):
     kw["workspace"] = _host((16,), "f32")
     kw["o"] = _host((2, 3, 40, 32))
     _expect_invalid(fa.fa_fwd_splitkv, "o must have shape", **kw)
+
+
+def _fp8(L, D=128, qd=1.0, kd=1.0, vd=1.0, Nq=16, q=1):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    f = ctypes.c_float
+    return L.fa_fwd_fp8(P(q), P(2), P(3), P(4), P(5), 1, 2, Nq, 64, D, 0, f(0.1), f(qd), f(kd), f(vd),
+                        None, None)
+
+
+def test_fp8_argument_errors_are_synchronous(L):
+    assert _fp8(L, D=64) == fa.FA_ERR_UNSUPPORTED
+    assert _fp8(L, D=96) == fa.FA_ERR_UNSUPPORTED
+    for bad in (0.0, -2.0, float("nan"), float("inf")):
+        assert _fp8(L, qd=bad) == fa.FA_ERR_INVALID_ARG
+        assert _fp8(L, kd=bad) == fa.FA_ERR_INVALID_ARG
+        assert _fp8(L, vd=bad) == fa.FA_ERR_INVALID_ARG
+    assert _fp8(L, qd=1e30, kd=1e30) == fa.FA_ERR_INVALID_ARG      # scale * descales overflows
+    assert _fp8(L, q=0) == fa.FA_ERR_INVALID_ARG
+    assert _fp8(L, Nq=0, q=None) == fa.FA_OK
+
+
+def test_fp8_binding_checks_types(L):
+    import torch
+    q = torch.zeros((1, 2, 8, 128), dtype=torch.float8_e4m3fn)
+    o = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    lse = torch.zeros((1, 2, 8), dtype=torch.float32)
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_fwd_fp8(q.to(torch.bfloat16), q, q, o, lse)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+    _expect_invalid(fa.fa_fwd_fp8, "o must be torch.bfloat16",
+                    q=q, k=q, v=q, o=o.to(torch.float16), lse=lse)
+    _expect_invalid(fa.fa_fwd_fp8, "v must be torch.float8_e4m3fn",
+                    q=q, k=q, v=q.to(torch.bfloat16), o=o, lse=lse)
+    _expect_invalid(fa.fa_fwd_fp8, "CUDA device", q=q, k=q, v=q, o=o, lse=lse)
