@@ -24,7 +24,7 @@ __all__ = [
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
     "lib", "library_path", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes",
     "fa_bwd_noalloc",
-    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_mask", "fa_bwd_mask",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "fa_profile_enable", "fa_profile_read",
@@ -66,6 +66,12 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd.restype = i
             L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, vp, vp]
             L.fa_fwd_fp8.restype = i
+            ll = ctypes.c_longlong
+            L.fa_fwd_mask.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, i, ll, vp]
+            L.fa_fwd_mask.restype = i
+            L.fa_bwd_mask.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                      vp, i, i, ll, vp, sz, vp]
+            L.fa_bwd_mask.restype = i
             L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
             L.fa_fwd_splitkv_workspace_bytes.restype = sz
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
@@ -218,6 +224,63 @@ def fa_fwd_fp8(q, k, v, o, lse, causal=False, scale=None, q_descale=1.0, k_desca
                           int(bool(causal)), float(scale), float(q_descale), float(k_descale),
                           float(v_descale), _ptr(key_bias), _stream_ptr(stream))
     _check(st, "fa_fwd_fp8")
+
+
+def _mask_args(what, mask, B, H, Nq, Nk, device):
+    """(mask_B, mask_H, ldm) of a general additive mask tensor: float32 of shape
+    [B or 1, H or 1, Nq, Nk] (or [Nq, Nk]) whose rows are contiguous and whose
+    row stride ldm is a multiple of 4 elements (a view of a [.., .., Nq, ldm]
+    buffer with ldm >= Nk is accepted), on the given device."""
+    import torch
+    if mask is None:
+        _bad(what, "mask is required")
+    m = mask if mask.dim() == 4 else mask.reshape(1, 1, *mask.shape) if mask.dim() == 2 else None
+    if m is None or tuple(m.shape[2:]) != (Nq, Nk) or m.shape[0] not in (1, B) or m.shape[1] not in (1, H):
+        _bad(what, f"mask must have shape [B or 1, H or 1, {Nq}, {Nk}], got {tuple(mask.shape)}")
+    if m.dtype != torch.float32:
+        _bad(what, f"mask must be torch.float32, got {m.dtype}")
+    Bm, Hm = int(m.shape[0]), int(m.shape[1])
+    ldm = int(m.stride(2)) if Nq > 1 else max(4, (Nk + 3) // 4 * 4)
+    if Nk > 0 and m.stride(3) != 1:
+        _bad(what, "mask rows must be contiguous")
+    if ldm < Nk or ldm % 4 != 0 or ldm < 4:
+        _bad(what, f"mask row stride must be >= Nk and a multiple of 4 elements, got {ldm}")
+    if (Hm > 1 and m.stride(1) != Nq * ldm) or (Bm > 1 and m.stride(0) != Hm * Nq * ldm):
+        _bad(what, "mask planes must be stored one after another")
+    if not m.is_cuda or m.device != device:
+        _bad(what, f"mask must be on {device}, got {m.device}")
+    if m.data_ptr() % 16 != 0:
+        _bad(what, "mask must start 16-byte aligned")
+    return Bm, Hm, ldm
+
+
+def fa_fwd_mask(q, k, v, o, lse, mask, causal=False, scale=None, stream=None):
+    """Forward with a general additive mask (see include/fa.h)."""
+    B, H, Nq, Nk, D, code = _validate("fa_fwd_mask", q, k, v, o=o, lse=lse, outputs=("o", "lse"))
+    Bm, Hm, ldm = _mask_args("fa_fwd_mask", mask, B, H, Nq, Nk, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    st = lib().fa_fwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
+                           int(bool(causal)), float(scale), code, _ptr(mask), Bm, Hm, ldm,
+                           _stream_ptr(stream))
+    _check(st, "fa_fwd_mask")
+
+
+def fa_bwd_mask(q, k, v, o, lse, dO, dq, dk, dv, workspace, mask, causal=False, scale=None,
+                stream=None):
+    """Backward with a general additive mask (see include/fa.h)."""
+    B, H, Nq, Nk, D, code = _validate("fa_bwd_mask", q, k, v, o=o, lse=lse, dO=dO, dq=dq, dk=dk,
+                                      dv=dv, workspace=workspace,
+                                      outputs=("o", "lse", "dO", "dq", "dk", "dv"))
+    Bm, Hm, ldm = _mask_args("fa_bwd_mask", mask, B, H, Nq, Nk, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_bwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                           _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)), float(scale),
+                           code, _ptr(mask), Bm, Hm, ldm, _ptr(workspace), nbytes,
+                           _stream_ptr(stream))
+    _check(st, "fa_bwd_mask")
 
 
 def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits) -> int:

@@ -285,6 +285,56 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+// Argument checks of the general mask (see fa_fwd_mask in fa.h).
+int check_mask(const float *mask, int B, int H, int Nq, int Nk, int mask_B, int mask_H, long long ldm) {
+    if (!mask || !aligned16(mask)) return FA_ERR_INVALID_ARG;
+    if ((mask_B != 1 && mask_B != B) || (mask_H != 1 && mask_H != H)) return FA_ERR_INVALID_ARG;
+    if (ldm < Nk || ldm < 4 || ldm % 4 != 0) return FA_ERR_INVALID_ARG;
+    const double elems = static_cast<double>(mask_B) * mask_H * Nq * static_cast<double>(ldm);
+    if (elems > 9.0e18) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                int Nq, int Nk, int D, int causal, float scale, int dtype, const float *mask,
+                int mask_B, int mask_H, long long ldm, void *stream) {
+    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (Nq == 0) return FA_OK;
+    if ((st = check_mask(mask, B, H, Nq, Nk, mask_B, mask_H, ldm)) != FA_OK) return st;
+    if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr, sms = 1;
+    if ((st = device_setup(dev, &err, &sms)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    const long long BH = static_cast<long long>(B) * H;
+    if (Nk == 0) {
+        return fa::launch_fwd_empty(o, lse, static_cast<size_t>(BH) * Nq, D, bf16, s) == cudaSuccess
+                   ? FA_OK : FA_ERR_CUDA;
+    }
+    fa::FwdTensorMaps tm;
+    if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
+    fa::FwdParams p = fwd_params(B, H, Nq, Nk, scale, nullptr, o, lse, err);
+    p.mask = mask;
+    p.mask_B = mask_B;
+    p.mask_H = mask_H;
+    p.ldm = ldm;
+    cudaError_t e = fa::launch_fwd_mask(tm, p, D, bf16, causal != 0, persistent_grid(p.n_units, sms), s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int D, int num_splits) {
     (void)Nk;
     if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128) || num_splits < 1 || num_splits > 256) return 0;
@@ -343,12 +393,18 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
     return up(rows * sizeof(float)) + 256;
 }
 
-int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-           const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
-           int causal, float scale, int dtype, const float *key_bias, void *workspace,
-           size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+// Shared body of fa_bwd and fa_bwd_mask (mask == nullptr: no general mask).
+int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
+             int causal, float scale, int dtype, const float *key_bias, const float *mask,
+             int mask_B, int mask_H, long long ldm, void *workspace, size_t workspace_bytes,
+             void *stream) {
     int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
     if (st != FA_OK) return st;
+    if (mask && Nq > 0 && (st = check_mask(mask, B, H, Nq, Nk, mask_B, mask_H, ldm)) != FA_OK) return st;
     if (Nq > 0 && (!q || !o || !lse || !dO || !dq)) return FA_ERR_INVALID_ARG;
     if (Nk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, key_bias, workspace};
@@ -385,6 +441,10 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
     p.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
     p.scale = scale;
     p.bias = key_bias;
+    p.mask = mask;
+    p.mask_B = mask_B;
+    p.mask_H = mask_H;
+    p.ldm = ldm;
     p.lse = lse;
     p.o = o;
     p.dO = dO;
@@ -401,8 +461,29 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
         if ((st = make_map(&tm.dv, dv, bf16, D, Nk, BH, 32)) != FA_OK) return st;
         if ((st = make_map(&tm.dq, dq, bf16, D, Nq, BH, 32)) != FA_OK) return st;
     }
-    cudaError_t e = fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
+    cudaError_t e = mask ? fa::launch_bwd_mask(tm, p, D, bf16, causal != 0, s)
+                         : fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
+           int causal, float scale, int dtype, const float *key_bias, void *workspace,
+           size_t workspace_bytes, void *stream) {
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, causal, scale, dtype, key_bias,
+                    nullptr, 0, 0, 0, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
+                int causal, float scale, int dtype, const float *mask, int mask_B, int mask_H,
+                long long ldm, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!mask) return FA_ERR_INVALID_ARG;
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, causal, scale, dtype, nullptr,
+                    mask, mask_B, mask_H, ldm, workspace, workspace_bytes, stream);
 }
 
 int fa_device_status(void *stream) {

@@ -12,6 +12,10 @@
 //   dS = P * (dP - D)  with D_i = sum_j P_ij dP_ij = rowsum(dO * O)
 //   dQ = scale dS K    dK = scale dS^T Q
 //
+// An optional additive term after scaling -- a per-key bias [B, Nk] or a
+// general mask [B or 1, H or 1, Nq, Nk] -- enters P exactly as in the forward
+// and receives no gradient.
+//
 // Three kernels on one stream, none of which stores S, P or dS:
 //   1. fa_bwd_pre_kernel   D_i = rowsum(dO * O) (fp32, the caller's workspace).
 //   2. fa_bwd_dkdv_kernel  one CTA per (b, h, 128-key tile); for every query
@@ -233,7 +237,7 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 //     dP^T(j+1)
 // so S^T(j+1) runs during phase 2 of j and dP^T(j+1) during phase 1 of j+1.
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -467,11 +471,24 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         float b2 = key < p.Nk ? 0.f : neg_inf();
         if (HAS_BIAS && key < p.Nk)
             b2 = __ldg(p.bias + static_cast<size_t>(bh / p.H) * p.Nk + key) * kLog2e;
+        // column `key` of the general mask: M[q][key] for the thread's queries
+        // (consecutive keys across the warp, so every load is one 128-byte line)
+        const float *mcol = nullptr;
+        if (HAS_MASK && key < p.Nk)
+            mcol = p.mask + mask_plane(bh, p.H, p.mask_B, p.mask_H) * p.Nq * p.ldm + key;
         bool ok = true;
         for (int jj = 0; jj < nq; ++jj) {
             const int s = jj & 1;
             const int qg = (j_begin + jj) * kBQ + 64 * g;     // first query of this thread's half
             const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256 + 64 * g;
+            float mk[HAS_MASK ? 64 : 1];
+            if constexpr (HAS_MASK) {
+                // issued before the wait for S^T so the loads overlap it
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    mk[e] = (mcol != nullptr && qg + e < p.Nq)
+                                ? __ldg(mcol + static_cast<long long>(qg + e) * p.ldm) * kLog2e : 0.f;
+            }
             // ---- phase 1: P^T = 2^(S^T qk + bias - LSE_2): registers (fp32) and
             // tensor memory (16-bit, the dV operand)
             {
@@ -495,8 +512,12 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int e4 = 0; e4 < 16; ++e4) {
                         const float4 lv = l4[e4];
                         // x = s qk + (bias - LSE_2), two columns per instruction
-                        const float2 c01 = __fadd2_rn(b22, make_float2(-lv.x, -lv.y));
-                        const float2 c23 = __fadd2_rn(b22, make_float2(-lv.z, -lv.w));
+                        float2 c01 = __fadd2_rn(b22, make_float2(-lv.x, -lv.y));
+                        float2 c23 = __fadd2_rn(b22, make_float2(-lv.z, -lv.w));
+                        if constexpr (HAS_MASK) {
+                            c01 = __fadd2_rn(c01, make_float2(mk[4 * e4], mk[4 * e4 + 1]));
+                            c23 = __fadd2_rn(c23, make_float2(mk[4 * e4 + 2], mk[4 * e4 + 3]));
+                        }
                         float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4]), __uint_as_float(sv[4 * e4 + 1])), qk2, c01);
                         float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])), qk2, c23);
                         if (!kEmu && diag) {
@@ -518,7 +539,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                 };
-                if (__all_sync(0xffffffffu, !HAS_BIAS && !diag && key < p.Nk))   // warp-uniform
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !diag && key < p.Nk))   // warp-uniform
                     make_p(std::true_type{});
                 else
                     make_p(std::false_type{});
@@ -623,7 +644,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 //     dQ(j)      once dS(j) is over the dP columns
 //     dP(j+1)    (over dS(j), read by dQ(j) just before, in order)
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -908,8 +929,31 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // last key this row may see
         const int lim = CAUSAL ? min(q + p.causal_off, p.Nk - 1) : p.Nk - 1;
+        // this row of the general mask (rows past Nq read nothing)
+        const float *mrow = nullptr;
+        if (HAS_MASK && q < p.Nq)
+            mrow = p.mask + (mask_plane(bh, p.H, p.mask_B, p.mask_H) * p.Nq + q) * p.ldm;
         for (int j = 0; j < n && ok; ++j) {
             const int kg = j * kBK + 64 * g;                  // first key of this thread's half
+            float mk[HAS_MASK ? 64 : 1];
+            if constexpr (HAS_MASK) {
+                // issued before the wait for S so the loads overlap it
+                if (mrow != nullptr && kg + 64 <= p.Nk) {
+                    const float4 *m4 = reinterpret_cast<const float4 *>(mrow + kg);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float4 mm = __ldg(m4 + e);
+                        mk[4 * e] = mm.x * kLog2e;
+                        mk[4 * e + 1] = mm.y * kLog2e;
+                        mk[4 * e + 2] = mm.z * kLog2e;
+                        mk[4 * e + 3] = mm.w * kLog2e;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        mk[e] = (mrow != nullptr && kg + e < p.Nk) ? __ldg(mrow + kg + e) * kLog2e : 0.f;
+                }
+            }
             {
                 const bool got = mbar_wait(bar(L::kSFull), j & 1, wctx);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -937,6 +981,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         float2 x;
                         if constexpr (HAS_BIAS)
                             x = __ffma2_rn(sc, qk2, __fadd2_rn(make_float2(bs[e], bs[e + 1]), nl2));
+                        else if constexpr (HAS_MASK)
+                            x = __ffma2_rn(sc, qk2, __fadd2_rn(make_float2(mk[e], mk[e + 1]), nl2));
                         else
                             x = __ffma2_rn(sc, qk2, nl2);
                         if (!kEmu && edge) {
@@ -953,7 +999,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     }
                 };
-                if (__all_sync(0xffffffffu, !HAS_BIAS && !edge && q < p.Nq))   // warp-uniform
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !edge && q < p.Nq))   // warp-uniform
                     make_p(std::true_type{});
                 else
                     make_p(std::false_type{});
@@ -1022,11 +1068,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
 cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
     {
         using L = DkdvLayout<D>;
-        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
@@ -1038,7 +1084,7 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
     }
     {
         using L = DqLayout<D>;
-        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS>;
+        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
@@ -1048,6 +1094,27 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
         note_launch();
         return cudaGetLastError();
     }
+}
+
+// 1. D_i = rowsum(dO * O) into the workspace
+template <int D, bool BF16>
+cudaError_t launch_pre(const BwdParams &p, cudaStream_t s) {
+    const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+    prof_begin(s, "fa_bwd_pre_kernel");
+    fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
+                                                     static_cast<const uint16_t *>(p.dO), p.Di, rows);
+    prof_end(s);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_mask_d(const BwdTensorMaps &tm, const BwdParams &p, bool causal, cudaStream_t s) {
+    cudaError_t e = launch_pre<D, BF16>(p, s);
+    if (e != cudaSuccess) return e;
+    return causal ? launch_grad_t<D, BF16, true, false, true>(tm, p, s)
+                  : launch_grad_t<D, BF16, false, false, true>(tm, p, s);
 }
 
 template <int D, bool BF16>
@@ -1072,6 +1139,14 @@ cudaError_t launch_bwd_d(const BwdTensorMaps &tm, const BwdParams &p, bool causa
 }
 
 }  // namespace
+
+cudaError_t launch_bwd_mask(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
+                            cudaStream_t stream) {
+    if (D == 64) return bf16 ? launch_bwd_mask_d<64, true>(tm, p, causal, stream)
+                             : launch_bwd_mask_d<64, false>(tm, p, causal, stream);
+    return bf16 ? launch_bwd_mask_d<128, true>(tm, p, causal, stream)
+                : launch_bwd_mask_d<128, false>(tm, p, causal, stream);
+}
 
 cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
                        bool has_bias, cudaStream_t stream) {

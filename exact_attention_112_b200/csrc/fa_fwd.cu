@@ -43,6 +43,9 @@
 //     = e^(s - m_new): l, o and the final LSE all use the same m_ref.
 //   * Causal: key tiles entirely above the diagonal are never loaded or
 //     multiplied; tiles crossing it are masked per element.
+//   * Additive terms after scaling: a per-key bias [B, Nk] (broadcast loads),
+//     or a general mask [B or 1, H or 1, Nq, Nk] whose row each softmax
+//     thread reads itself (the "+ mask" of the SDPA formula in full).
 //   * Epilogue: each softmax thread divides its O row by l and stores it
 //     straight from registers (so the Q buffer is free for the next unit).
 //
@@ -103,7 +106,6 @@ struct FwdLayout {
     static constexpr int kKSteps = kRowBytes / 32;        // MMA K-steps of S (32 bytes each)
     static constexpr int kPvKeys = 32 / kElemBytes;       // keys per P.V instruction
     static constexpr int kPvSteps = kBN / kPvKeys;        // P.V instructions per tile
-    static constexpr int kPCols = kBN * kElemBytes / 4;   // tensor-memory columns of P
     static constexpr int kQ = 0;                          // 2 tiles
     static constexpr int kK = kQ + 2 * kTileBytes;        // kStages tiles
     static constexpr int kV = kK + kStages * kTileBytes;  // kStages tiles
@@ -204,11 +206,13 @@ __device__ __forceinline__ bool next_work(const FwdParams &p, int &r, Unit &w) {
     }
 }
 
-template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false>
+template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false, bool HAS_MASK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using L = FwdLayout<D, ELEM>;
+    // scores arrive already scaled (and offset) when an additive term is present
+    constexpr bool kAdd = HAS_BIAS || HAS_MASK;
     constexpr bool kFp8 = ELEM == kElemE4M3;
     constexpr bool kOutBF16 = ELEM != kElemF16;   // O storage type
     extern __shared__ uint8_t smem_raw[];
@@ -484,6 +488,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // last key index this row may see
             const int lim = CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1;
             const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(w.bh / p.H) * p.Nk : nullptr;
+            // this row of the general mask (rows past Nq read nothing)
+            const float *mrow = nullptr;
+            if (HAS_MASK && qrow < p.Nq)
+                mrow = p.mask + (mask_plane(w.bh, p.H, p.mask_B, p.mask_H) * p.Nq + qrow) * p.ldm;
             float m_ref = neg_inf();   // log2 units
             float l = 0.f;
             for (int j = 0; j < w.n_kv; ++j, ++t) {
@@ -518,6 +526,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             x[c] = fmaf(__uint_as_float(sr[c]), qk, bb);
                         }
                     }
+                } else if constexpr (HAS_MASK) {
+                    // x = s * qk_scale + M_ij * log2(e); the thread reads its own
+                    // row (512 contiguous bytes per tile, L1-cached)
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    if (mrow != nullptr && kv0 + kBN <= p.Nk) {
+                        const float4 *m4 = reinterpret_cast<const float4 *>(mrow + kv0);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const float4 mm = __ldg(m4 + c);
+                            x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, mm.x * kLog2e);
+                            x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, mm.y * kLog2e);
+                            x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, mm.z * kLog2e);
+                            x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, mm.w * kLog2e);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c) {
+                            const float mm = (mrow != nullptr && kv0 + c < p.Nk) ? __ldg(mrow + kv0 + c) * kLog2e : 0.f;
+                            x[c] = fmaf(__uint_as_float(sr[c]), qk, mm);
+                        }
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
@@ -527,16 +556,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int c = 0; c < 128; ++c)
                         if (kv0 + c > lim) x[c] = neg_inf();
                 }
+                // row maximum: four independent chains of three-input maxima
                 float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
 #pragma unroll
-                for (int c = 4; c < 128; c += 4) {
-                    mx0 = fmaxf(mx0, x[c]);
-                    mx1 = fmaxf(mx1, x[c + 1]);
-                    mx2 = fmaxf(mx2, x[c + 2]);
-                    mx3 = fmaxf(mx3, x[c + 3]);
+                for (int c = 4; c < 124; c += 8) {
+                    mx0 = fmax3(mx0, x[c], x[c + 1]);
+                    mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+                    mx2 = fmax3(mx2, x[c + 4], x[c + 5]);
+                    mx3 = fmax3(mx3, x[c + 6], x[c + 7]);
                 }
-                float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-                if constexpr (!HAS_BIAS) m_tile *= qk;   // qk > 0: max commutes with scaling
+                float m_tile = fmax3(fmax3(mx0, mx1, x[124]), fmax3(mx2, mx3, x[125]), fmaxf(x[126], x[127]));
+                if constexpr (!kAdd) m_tile *= qk;   // qk > 0: max commutes with scaling
                 const bool need = m_tile > m_ref + kTau;
                 // warp-uniform: if any row of the warp moves its reference maximum,
                 // the warp rescales its O rows (before the first half of P is
@@ -552,13 +582,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
                 // p = 2^(x - m), two columns per paired-fp32 instruction, in two
                 // halves of 64 keys; each half goes back over the S columns and
-                // is handed to the MMA warp on its own barrier.  On tiles without
-                // masked scores, one pair in kEmuEvery goes through the FMA-pipe
-                // exponential instead of MUFU.
-                float2 lsum = make_float2(0.f, 0.f);
+                // is handed to the MMA warp on its own barrier.  One pair in
+                // kEmuEvery goes through the FMA-pipe exponential instead of MUFU
+                // once every row of the warp has a finite reference maximum: a
+                // masked score (-inf) then yields 2^-126 instead of 0, which is
+                // invisible next to l >= 1 (the score that set m_ref contributes
+                // 2^(m_tile - m_ref) >= 1); rows that have seen no key yet keep
+                // the exact MUFU path so that they still end with l = 0.
+                float2 lsum = make_float2(0.f, 0.f), lsum2 = make_float2(0.f, 0.f);
                 const float2 neg_m2 = make_float2(-m_use, -m_use);
                 const float2 qk2 = make_float2(qk, qk);
-                const bool emu = __all_sync(0xffffffffu, !HAS_BIAS && kv0 + kBN - 1 <= lim);   // warp-uniform
+                const bool emu = __all_sync(0xffffffffu, m_ref != neg_inf());   // warp-uniform
                 auto half = [&](int h, auto emu_tag) {
                     constexpr bool kEmu = decltype(emu_tag)::value;
                     float pv[64];
@@ -566,13 +600,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int c2 = 0; c2 < 32; ++c2) {
                         const int c = 64 * h + 2 * c2;
                         const float2 xc = make_float2(x[c], x[c + 1]);
-                        const float2 a = HAS_BIAS ? __fadd2_rn(xc, neg_m2) : __ffma2_rn(xc, qk2, neg_m2);
+                        const float2 a = kAdd ? __fadd2_rn(xc, neg_m2) : __ffma2_rn(xc, qk2, neg_m2);
                         float2 pp;
                         if (kEmu && c2 % kEmuEvery == kEmuEvery - 1)
                             pp = exp2_fma2(a);
                         else
                             pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-                        lsum = __fadd2_rn(lsum, pp);
+                        if (c2 & 1)
+                            lsum2 = __fadd2_rn(lsum2, pp);
+                        else
+                            lsum = __fadd2_rn(lsum, pp);
                         pv[2 * c2] = pp.x;
                         pv[2 * c2 + 1] = pp.y;
                     }
@@ -617,7 +654,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(L::kPHalf + 2 * i + 1));
-                l += lsum.x + lsum.y;
+                l += (lsum.x + lsum.y) + (lsum2.x + lsum2.y);
             }
             if (!ok) break;
 
@@ -750,6 +787,20 @@ cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, 
     return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool CAUSAL>
+cudaError_t launch_mask_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
+    constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
+    using L = FwdLayout<D, kElem>;
+    auto kern = fa_fwd_kernel<D, kElem, CAUSAL, false, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    prof_begin(stream, "fa_fwd_mask_kernel");
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    prof_end(stream);
+    note_launch();
+    return cudaGetLastError();
+}
+
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
     constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
@@ -795,6 +846,16 @@ cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, int e
                                           : launch_fwd_d<64, kElemF16>(tm, p, causal, has_bias, grid, stream);
     return elem == kElemBF16 ? launch_fwd_d<128, kElemBF16>(tm, p, causal, has_bias, grid, stream)
                              : launch_fwd_d<128, kElemF16>(tm, p, causal, has_bias, grid, stream);
+}
+
+cudaError_t launch_fwd_mask(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                            int grid, cudaStream_t stream) {
+    if (D == 64) {
+        if (bf16) return causal ? launch_mask_t<64, true, true>(tm, p, grid, stream) : launch_mask_t<64, true, false>(tm, p, grid, stream);
+        return causal ? launch_mask_t<64, false, true>(tm, p, grid, stream) : launch_mask_t<64, false, false>(tm, p, grid, stream);
+    }
+    if (bf16) return causal ? launch_mask_t<128, true, true>(tm, p, grid, stream) : launch_mask_t<128, true, false>(tm, p, grid, stream);
+    return causal ? launch_mask_t<128, false, true>(tm, p, grid, stream) : launch_mask_t<128, false, false>(tm, p, grid, stream);
 }
 
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,

@@ -21,6 +21,9 @@ struct FwdParams {
     float qk_scale_log2;           // scale * log2(e) (E4M3: times the Q and K descales)
     float o_scale;                 // multiplies O = o / l at the end (E4M3: the V descale)
     const float *bias;             // [B, Nk] or nullptr
+    const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
+    int mask_B, mask_H;            // 1 (broadcast) or B, H
+    long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
     void *o;                       // [B*H, Nq, D] 16-bit output
     float *lse;                    // [B*H, Nq]
     int *err;                      // device error word
@@ -43,6 +46,9 @@ struct BwdParams {
     float qk_scale_log2;           // scale * log2(e)
     float scale;
     const float *bias;             // [B, Nk] or nullptr
+    const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
+    int mask_B, mask_H;            // 1 (broadcast) or B, H
+    long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
     const float *lse;              // [B*H, Nq] from the forward
     const void *o, *dO;            // [B*H, Nq, D] 16-bit
     float *Di;                     // workspace: [B*H*Nq]
@@ -56,6 +62,15 @@ struct BwdTensorMaps {
 
 cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
                        bool has_bias, cudaStream_t stream);
+// Backward with the general additive mask p.mask (no key bias).
+cudaError_t launch_bwd_mask(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
+                            cudaStream_t stream);
+
+// Plane of the general mask used by head bh (b = bh / H, h = bh % H).
+__host__ __device__ inline long long mask_plane(int bh, int H, int mask_B, int mask_H) {
+    const int b = bh / H, h = bh % H;
+    return static_cast<long long>(mask_B > 1 ? b : 0) * mask_H + (mask_H > 1 ? h : 0);
+}
 
 // Counts every kernel launch made by the library (fa_launch_count()).
 void note_launch(unsigned n = 1);
@@ -69,6 +84,9 @@ void prof_end(cudaStream_t stream);
 // work units in a fixed snake order.
 cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, int elem, bool causal,
                        bool has_bias, int grid, cudaStream_t stream);
+// Forward with the general additive mask p.mask (16-bit inputs, no key bias).
+cudaError_t launch_fwd_mask(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                            int grid, cudaStream_t stream);
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                              bool has_bias, int grid, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,

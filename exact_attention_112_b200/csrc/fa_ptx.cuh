@@ -363,8 +363,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // p(0) = 1 whose coefficients were fitted for this library by minimising the
 // maximum relative error on [-1/2, 1/2] (1.03e-4; P is then rounded to
 // 16 bits, a 2^-9 step); 2^n is added to the exponent field.  Valid for
-// x <= 127; x below -126 is clamped to -126 (2^-126 instead of a smaller
-// value), so callers use it only where no score is masked to -inf.
+// x <= 127; x below -126 (a masked score, -inf, included) is clamped to -126,
+// giving 2^-126 instead of a smaller value or 0, so callers use it only where
+// such a term is negligible against the row sum (never for a row that may end
+// with no visible key).
 __device__ __forceinline__ float2 exp2_fma2(float2 x) {
     constexpr float kShift = 12582912.f;   // 1.5 * 2^23
     constexpr float c1 = 6.932791870e-01f, c2 = 2.422159912e-01f, c3 = 5.503048995e-02f;
@@ -379,6 +381,13 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
     // to the exponent of q (the shifter's own bits move out of the word)
     return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
                        __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+}
+
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ float lg2_approx(float x) {

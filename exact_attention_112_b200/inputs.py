@@ -110,6 +110,57 @@ def make_key_bias(B, Nk, frac, seed):
     return bias
 
 
+def make_mask(kind, Nq, Nk, seed, planes=(1, 1), ldm=None):
+    """General additive mask, float32 [Bm, Hm, Nq, ldm] (columns [Nk, ldm) are
+    padding, filled with NaN so that reading them would show; the mask proper
+    is the [..., :Nk] view, which is returned).  Kinds:
+      random    -inf on a seeded 10% of entries, elsewhere N(0, 0.5^2) values;
+                every row keeps its first visible key finite, so no row is
+                fully hidden
+      window    sliding window: key j visible to query i iff
+                i' - 255 <= j <= i' with i' = i + Nk - Nq (bottom-right)
+      document  packed documents of seeded lengths 1..max(1, Nk // 3):
+                causal inside a document, hidden across documents (query
+                rows are aligned to the keys bottom-right)
+      rows      like random, and every 7th query row entirely -inf (rows
+                that see no key: O = 0, LSE = -inf)
+    """
+    Bm, Hm = planes
+    if ldm is None:
+        ldm = max(4, (Nk + 3) // 4 * 4)
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    buf = torch.full((Bm, Hm, Nq, ldm), float("nan"), dtype=torch.float32)
+    m = buf[..., :Nk]
+    i = torch.arange(Nq).view(-1, 1) + (Nk - Nq)
+    j = torch.arange(Nk).view(1, -1)
+    if kind in ("random", "rows"):
+        vals = torch.randn((Bm, Hm, Nq, Nk), generator=gen) * 0.5
+        hide = torch.rand((Bm, Hm, Nq, Nk), generator=gen) < 0.1
+        if Nk > 0:
+            hide[..., 0] = False
+        vals[hide] = -math.inf
+        if kind == "rows":
+            vals[:, :, ::7, :] = -math.inf
+        m.copy_(vals)
+    elif kind == "window":
+        vis = (j <= i) & (j >= i - 255)
+        m.copy_(torch.where(vis, 0.0, -math.inf).expand(Bm, Hm, Nq, Nk))
+    elif kind == "document":
+        doc = torch.empty(Nk, dtype=torch.long)
+        start, d = 0, 0
+        while start < Nk:
+            ln = int(torch.randint(1, max(2, Nk // 3 + 1), (1,), generator=gen))
+            doc[start:start + ln] = d
+            start += ln
+            d += 1
+        qdoc = doc[torch.clamp(i.view(-1), 0, max(Nk - 1, 0))].view(-1, 1) if Nk > 0 else None
+        vis = (j <= i) & (qdoc == doc.view(1, -1)) if Nk > 0 else torch.zeros((Nq, 0), dtype=torch.bool)
+        m.copy_(torch.where(vis, 0.0, -math.inf).expand(Bm, Hm, Nq, Nk))
+    else:
+        raise ValueError(kind)
+    return m
+
+
 def sample_rows(N, n_random=512, tile=128, seed=0):
     """Query rows checked at full size: every tile-boundary row (0, 127, 128,
     255, ..., N-1) plus n_random seeded rows, sorted and unique."""

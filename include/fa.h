@@ -141,6 +141,33 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            size_t workspace_bytes, void *stream);
 
 /*
+ * Forward and backward with a general additive mask: the "+ mask" of the SDPA
+ * formula in full ("Attention is where tokens meet"),
+ *     S = scale * Q K^T + M,   O = softmax(S) V,
+ * with M a float32 [mask_B, mask_H, Nq, ldm] array in device memory (row i,
+ * columns [0, Nk) of plane (b, h) are M_ij for batch b, head h):
+ *   mask_B   1 (the same planes for every batch) or B;
+ *   mask_H   1 (the same plane for every head) or H;
+ *   ldm      row stride in elements: ldm >= Nk, a multiple of 4 (rows start
+ *            16-byte aligned); columns [Nk, ldm) are never read.
+ * Entries are finite or -inf (-inf = key hidden from that query).  causal may
+ * be combined with the mask; there is no separate key bias (fold it into M).
+ * A row whose keys are all hidden gets O = 0 and LSE = -inf.  The mask
+ * receives no gradient.  Arguments, layouts and results are otherwise those
+ * of fa_fwd() and fa_bwd(); the mask adds Nq * Nk * 4 bytes of reads per
+ * plane, so these calls are bound by memory bandwidth rather than the tensor
+ * cores.  Invalid mask arguments return FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int Nq, int Nk, int D, int causal, float scale, int dtype,
+                const float *mask, int mask_B, int mask_H, long long ldm, void *stream);
+int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o,
+                const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                int B, int H, int Nq, int Nk, int D, int causal, float scale,
+                int dtype, const float *mask, int mask_B, int mask_H, long long ldm,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Largest B * H * Nq that fa_bwd_noalloc() accepts.
  */
 #define FA_BWD_NOALLOC_MAX_ROWS 1048576
