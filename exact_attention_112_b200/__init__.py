@@ -25,6 +25,7 @@ __all__ = [
     "lib", "library_path", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes",
     "fa_bwd_noalloc",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_mask", "fa_bwd_mask",
+    "fa_fwd_varlen", "fa_bwd_varlen",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "fa_profile_enable", "fa_profile_read",
@@ -72,6 +73,11 @@ def lib() -> ctypes.CDLL:
             L.fa_bwd_mask.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
                                       vp, i, i, ll, vp, sz, vp]
             L.fa_bwd_mask.restype = i
+            L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
+            L.fa_fwd_varlen.restype = i
+            L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                        i, i, f, i, vp, sz, vp]
+            L.fa_bwd_varlen.restype = i
             L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
             L.fa_fwd_splitkv_workspace_bytes.restype = sz
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
@@ -281,6 +287,66 @@ def fa_bwd_mask(q, k, v, o, lse, dO, dq, dk, dv, workspace, mask, causal=False, 
                            code, _ptr(mask), Bm, Hm, ldm, _ptr(workspace), nbytes,
                            _stream_ptr(stream))
     _check(st, "fa_bwd_mask")
+
+
+def _varlen_args(what, q, k, cu_q, cu_k, max_q, max_k):
+    """Shapes of the packed layout: q [H, total_q, D], k [H, total_k, D], the
+    int32 sequence tables [num_seqs + 1] on q's device."""
+    import torch
+    if q is None or q.dim() != 3 or k is None or k.dim() != 3:
+        _bad(what, "packed q and k must be 3-D tensors [H, total, D]")
+    H, total_q, D = q.shape
+    if k.shape[0] != H or k.shape[2] != D:
+        _bad(what, f"k must be [H={H}, total_k, D={D}], got {tuple(k.shape)}")
+    for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
+        if t is None or t.dim() != 1 or t.dtype != torch.int32 or not t.is_contiguous():
+            _bad(what, f"{name} must be a contiguous int32 vector [num_seqs + 1]")
+        if not t.is_cuda or t.device != q.device:
+            _bad(what, f"{name} must be on {q.device}")
+    if cu_q.numel() != cu_k.numel() or cu_q.numel() < 2:
+        _bad(what, "cu_seqlens_q and cu_seqlens_k must both have num_seqs + 1 >= 2 entries")
+    if int(max_q) < 0 or int(max_k) < 0:
+        _bad(what, "max_seqlen_q and max_seqlen_k must be >= 0")
+    return int(cu_q.numel() - 1), H, total_q, int(k.shape[1]), D
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                  causal=False, scale=None, stream=None):
+    """Forward of packed variable-length sequences (see include/fa.h): q, o
+    [H, total_q, D], k, v [H, total_k, D], lse [H, total_q]."""
+    nseq, H, tq, tk, D = _varlen_args("fa_fwd_varlen", q, k, cu_seqlens_q, cu_seqlens_k,
+                                      max_seqlen_q, max_seqlen_k)
+    # the packed tensors are the fixed layout with B = 1 and N = total
+    _, _, _, _, _, code = _validate("fa_fwd_varlen", q[None], k[None], v[None] if v is not None else None,
+                                    o=None if o is None else o[None],
+                                    lse=None if lse is None else lse[None], outputs=("o", "lse"))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    st = lib().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                             _ptr(cu_seqlens_k), nseq, H, tq, tk, int(max_seqlen_q),
+                             int(max_seqlen_k), D, int(bool(causal)), float(scale), code,
+                             _stream_ptr(stream))
+    _check(st, "fa_fwd_varlen")
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k,
+                  max_seqlen_q, max_seqlen_k, causal=False, scale=None, stream=None):
+    """Backward of packed variable-length sequences (see include/fa.h)."""
+    nseq, H, tq, tk, D = _varlen_args("fa_bwd_varlen", q, k, cu_seqlens_q, cu_seqlens_k,
+                                      max_seqlen_q, max_seqlen_k)
+    add = lambda t: None if t is None else t[None]
+    _, _, _, _, _, code = _validate("fa_bwd_varlen", q[None], k[None], add(v), o=add(o), lse=add(lse),
+                                    dO=add(dO), dq=add(dq), dk=add(dk), dv=add(dv),
+                                    workspace=workspace,
+                                    outputs=("o", "lse", "dO", "dq", "dk", "dv"))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), nseq, H,
+                             tq, tk, int(max_seqlen_q), int(max_seqlen_k), D, int(bool(causal)),
+                             float(scale), code, _ptr(workspace), nbytes, _stream_ptr(stream))
+    _check(st, "fa_bwd_varlen")
 
 
 def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits) -> int:

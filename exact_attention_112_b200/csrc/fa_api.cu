@@ -212,6 +212,8 @@ fa::FwdParams fwd_params(int B, int H, int Nq, int Nk, float scale, const float 
     p.timeout_ns = kDefaultTimeoutNs;
     p.num_splits = 1;
     p.tiles_per_split = 0;
+    p.cu_q = p.cu_k = nullptr;
+    p.total_q = p.total_k = 0;
     return p;
 }
 }  // namespace
@@ -335,6 +337,59 @@ int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+// Argument checks of the packed variable-length entry points.
+int check_varlen(const int *cu_q, const int *cu_k, int num_seqs, int H, int total_q, int total_k,
+                 int max_q, int max_k, int D, int causal, float scale, int dtype) {
+    int st = check_common(num_seqs, H, max_q, max_k, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (!cu_q || !cu_k || (reinterpret_cast<uintptr_t>(cu_q) & 3) || (reinterpret_cast<uintptr_t>(cu_k) & 3))
+        return FA_ERR_INVALID_ARG;
+    if (total_q < 0 || total_k < 0 || total_q > (1 << 30) || total_k > (1 << 30)) return FA_ERR_INVALID_ARG;
+    if (static_cast<long long>(H) * total_q > INT32_MAX || static_cast<long long>(H) * total_k > INT32_MAX)
+        return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens_q, const int *cu_seqlens_k, int num_seqs, int H, int total_q,
+                  int total_k, int max_seqlen_q, int max_seqlen_k, int D, int causal, float scale,
+                  int dtype, void *stream) {
+    int st = check_varlen(cu_seqlens_q, cu_seqlens_k, num_seqs, H, total_q, total_k, max_seqlen_q,
+                          max_seqlen_k, D, causal, scale, dtype);
+    if (st != FA_OK) return st;
+    if (total_q == 0 || max_seqlen_q == 0) return FA_OK;
+    if (!q || !o || !lse || (total_k > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr, sms = 1;
+    if ((st = device_setup(dev, &err, &sms)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == FA_BF16;
+    if (total_k == 0 || max_seqlen_k == 0) {
+        return fa::launch_fwd_empty(o, lse, static_cast<size_t>(H) * total_q, D, bf16, s) == cudaSuccess
+                   ? FA_OK : FA_ERR_CUDA;
+    }
+    fa::FwdTensorMaps tm;
+    if ((st = make_map(&tm.q, q, bf16, D, total_q, H, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.k, k, bf16, D, total_k, H, 128)) != FA_OK) return st;
+    if ((st = make_map(&tm.v, v, bf16, D, total_k, H, 128)) != FA_OK) return st;
+    fa::FwdParams p = fwd_params(num_seqs, H, max_seqlen_q, max_seqlen_k, scale, nullptr, o, lse, err);
+    p.cu_q = cu_seqlens_q;
+    p.cu_k = cu_seqlens_k;
+    p.total_q = total_q;
+    p.total_k = total_k;
+    cudaError_t e = fa::launch_fwd_varlen(tm, p, D, bf16, causal != 0, persistent_grid(p.n_units, sms), s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int D, int num_splits) {
     (void)Nk;
     if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128) || num_splits < 1 || num_splits > 256) return 0;
@@ -397,20 +452,34 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
 
 namespace {
 // Shared body of fa_bwd and fa_bwd_mask (mask == nullptr: no general mask).
+// Packed variable-length sequences of the backward (cu_q == nullptr: fixed layout).
+struct VarlenArgs {
+    const int *cu_q = nullptr, *cu_k = nullptr;
+    int total_q = 0, total_k = 0;
+};
+
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
              int causal, float scale, int dtype, const float *key_bias, const float *mask,
              int mask_B, int mask_H, long long ldm, void *workspace, size_t workspace_bytes,
-             void *stream) {
-    int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
+             void *stream, const VarlenArgs &vl = VarlenArgs{}) {
+    const bool varlen = vl.cu_q != nullptr;
+    int st = varlen ? check_varlen(vl.cu_q, vl.cu_k, B, H, vl.total_q, vl.total_k, Nq, Nk, D, causal, scale, dtype)
+                    : check_common(B, H, Nq, Nk, D, causal, scale, dtype);
     if (st != FA_OK) return st;
+    // rows of the q-side and k-side tensors: [B*H, N] or, packed, [H, total]
+    const long long q_rows = varlen ? static_cast<long long>(H) * vl.total_q : static_cast<long long>(B) * H * Nq;
+    const long long k_rows = varlen ? static_cast<long long>(H) * vl.total_k : static_cast<long long>(B) * H * Nk;
+    if (varlen && (vl.total_q == 0 || Nq == 0)) Nq = 0;
+    if (varlen && (vl.total_k == 0 || Nk == 0)) Nk = 0;
     if (mask && Nq > 0 && (st = check_mask(mask, B, H, Nq, Nk, mask_B, mask_H, ldm)) != FA_OK) return st;
     if (Nq > 0 && (!q || !o || !lse || !dO || !dq)) return FA_ERR_INVALID_ARG;
     if (Nk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, key_bias, workspace};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
-    const size_t need = fa_bwd_workspace_bytes(B, H, Nq, Nk, D);
+    const size_t need = varlen ? fa_bwd_workspace_bytes(1, H, vl.total_q, vl.total_k, D)
+                               : fa_bwd_workspace_bytes(B, H, Nq, Nk, D);
     if (Nq > 0 && (!workspace || workspace_bytes < need)) return FA_ERR_WORKSPACE;
     int dev;
     if ((st = current_device(&dev)) != FA_OK) return st;
@@ -421,15 +490,15 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     const long long BH = static_cast<long long>(B) * H;
     if (Nq == 0) {
         // no query: every key and value gradient is zero
-        if (Nk == 0) return FA_OK;
-        const size_t bytes = static_cast<size_t>(BH) * Nk * D * 2;
+        if (Nk == 0 || k_rows == 0) return FA_OK;
+        const size_t bytes = static_cast<size_t>(k_rows) * D * 2;
         if (cudaMemsetAsync(dk, 0, bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, s) != cudaSuccess)
             return FA_ERR_CUDA;
         return FA_OK;
     }
     if (Nk == 0) {
         // no key: every output row is empty, so dQ is zero
-        if (cudaMemsetAsync(dq, 0, static_cast<size_t>(BH) * Nq * D * 2, s) != cudaSuccess) return FA_ERR_CUDA;
+        if (cudaMemsetAsync(dq, 0, static_cast<size_t>(q_rows) * D * 2, s) != cudaSuccess) return FA_ERR_CUDA;
         return FA_OK;
     }
     fa::BwdParams p;
@@ -448,20 +517,31 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     p.lse = lse;
     p.o = o;
     p.dO = dO;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
     p.Di = static_cast<float *>(workspace);
     p.err = err;
     p.timeout_ns = kDefaultTimeoutNs;
+    p.cu_q = vl.cu_q;
+    p.cu_k = vl.cu_k;
+    p.total_q = vl.total_q;
+    p.total_k = vl.total_k;
+    // tensor maps over [B*H, N, D] or, packed, [H, total, D]
+    const int nq_map = varlen ? vl.total_q : Nq, nk_map = varlen ? vl.total_k : Nk;
+    const long long z_map = varlen ? H : BH;
     fa::BwdTensorMaps tm;
     {
-        if ((st = make_map(&tm.q, q, bf16, D, Nq, BH, 128)) != FA_OK) return st;
-        if ((st = make_map(&tm.dO, dO, bf16, D, Nq, BH, 128)) != FA_OK) return st;
-        if ((st = make_map(&tm.k, k, bf16, D, Nk, BH, 128)) != FA_OK) return st;
-        if ((st = make_map(&tm.v, v, bf16, D, Nk, BH, 128)) != FA_OK) return st;
-        if ((st = make_map(&tm.dk, dk, bf16, D, Nk, BH, 32)) != FA_OK) return st;
-        if ((st = make_map(&tm.dv, dv, bf16, D, Nk, BH, 32)) != FA_OK) return st;
-        if ((st = make_map(&tm.dq, dq, bf16, D, Nq, BH, 32)) != FA_OK) return st;
+        if ((st = make_map(&tm.q, q, bf16, D, nq_map, z_map, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.dO, dO, bf16, D, nq_map, z_map, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.k, k, bf16, D, nk_map, z_map, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.v, v, bf16, D, nk_map, z_map, 128)) != FA_OK) return st;
+        if ((st = make_map(&tm.dk, dk, bf16, D, nk_map, z_map, 32)) != FA_OK) return st;
+        if ((st = make_map(&tm.dv, dv, bf16, D, nk_map, z_map, 32)) != FA_OK) return st;
+        if ((st = make_map(&tm.dq, dq, bf16, D, nq_map, z_map, 32)) != FA_OK) return st;
     }
-    cudaError_t e = mask ? fa::launch_bwd_mask(tm, p, D, bf16, causal != 0, s)
+    cudaError_t e = varlen ? fa::launch_bwd_varlen(tm, p, D, bf16, causal != 0, s)
+                  : mask ? fa::launch_bwd_mask(tm, p, D, bf16, causal != 0, s)
                          : fa::launch_bwd(tm, p, D, bf16, causal != 0, key_bias != nullptr, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -475,6 +555,21 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            size_t workspace_bytes, void *stream) {
     return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, causal, scale, dtype, key_bias,
                     nullptr, 0, 0, 0, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dO, void *dq, void *dk, void *dv, const int *cu_seqlens_q,
+                  const int *cu_seqlens_k, int num_seqs, int H, int total_q, int total_k,
+                  int max_seqlen_q, int max_seqlen_k, int D, int causal, float scale, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream) {
+    if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+    VarlenArgs vl;
+    vl.cu_q = cu_seqlens_q;
+    vl.cu_k = cu_seqlens_k;
+    vl.total_q = total_q;
+    vl.total_k = total_k;
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, num_seqs, H, max_seqlen_q, max_seqlen_k, D, causal,
+                    scale, dtype, nullptr, nullptr, 0, 0, 0, workspace, workspace_bytes, stream, vl);
 }
 
 int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o, const float *lse,

@@ -12,6 +12,9 @@
 //   dS = P * (dP - D)  with D_i = sum_j P_ij dP_ij = rowsum(dO * O)
 //   dQ = scale dS K    dK = scale dS^T Q
 //
+// Packed variable-length sequences (VARLEN instances) read each (sequence,
+// head)'s rows through seq_rows() and store dQ, dK, dV row by row.
+//
 // An optional additive term after scaling -- a per-key bias [B, Nk] or a
 // general mask [B or 1, H or 1, Nq, Nk] -- enters P exactly as in the forward
 // and receives no gradient.
@@ -237,7 +240,7 @@ __device__ __forceinline__ void stage_row_sw128(uint8_t *tile, int row, int col0
 //     dP^T(j+1)
 // so S^T(j+1) runs during phase 2 of j and dP^T(j+1) during phase 1 of j+1.
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false, bool VARLEN = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -264,10 +267,17 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int t, bh;   // key tile 0 is seen by the most query tiles
     unit_of(blockIdx.x, BH, (p.Nk + kBK - 1) / kBK, t, bh);
     const int kv0 = t * kBK;
-    const int n_q_all = (p.Nq + kBQ - 1) / kBQ;
+    // rows of this (sequence, head): fixed [B*H, N, D] layout or packed sequences
+    const SeqRows sr = VARLEN ? seq_rows(bh, p.H, p.Nq, p.Nk, p.cu_q, p.cu_k, p.total_q, p.total_k)
+                              : SeqRows{static_cast<long long>(bh) * p.Nq, static_cast<long long>(bh) * p.Nk, p.Nq, p.Nk};
+    const int len_q = sr.len_q, len_k = sr.len_k, coff = len_k - len_q;
+    const int q_y0 = VARLEN ? static_cast<int>(sr.q_row0 - static_cast<long long>(bh % p.H) * p.total_q) : 0;
+    const int k_y0 = VARLEN ? static_cast<int>(sr.k_row0 - static_cast<long long>(bh % p.H) * p.total_k) : 0;
+    const int z = VARLEN ? bh % p.H : bh;           // head slice of the tensor maps
+    const int n_q_all = kv0 < len_k ? (len_q + kBQ - 1) / kBQ : 0;   // a tile past the keys: no work
     int j_begin = 0;
     if (CAUSAL) {
-        const int first_q = kv0 - p.causal_off;      // first query that sees key kv0
+        const int first_q = kv0 - coff;              // first query that sees key kv0
         j_begin = first_q > 0 ? first_q / kBQ : 0;
         if (j_begin > n_q_all) j_begin = n_q_all;
     }
@@ -309,15 +319,15 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp >= 8) regs_release<kRegsOther>();
     if (warp == kProducerWarp) {
         // ===================== producer =====================
-        const float *lse_bh = p.lse + static_cast<size_t>(bh) * p.Nq;
-        const float *di_bh = p.Di + static_cast<size_t>(bh) * p.Nq;
+        const float *lse_bh = p.lse + sr.q_row0;
+        const float *di_bh = p.Di + sr.q_row0;
         bool ok = true;
         int issued = 0;
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(L::kKVFull), 2 * L::kTileBytes);
             for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(sbase + L::kK + c * L::kChunkBytes, &tm_k, bar(L::kKVFull), c * 64, kv0, bh);
-                tma_load_3d(sbase + L::kV + c * L::kChunkBytes, &tm_v, bar(L::kKVFull), c * 64, kv0, bh);
+                tma_load_3d(sbase + L::kK + c * L::kChunkBytes, &tm_k, bar(L::kKVFull), c * 64, k_y0 + kv0, z);
+                tma_load_3d(sbase + L::kV + c * L::kChunkBytes, &tm_v, bar(L::kKVFull), c * 64, k_y0 + kv0, z);
             }
         }
         for (int jj = 0; jj < nq; ++jj) {
@@ -330,9 +340,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 mbar_arrive_expect_tx(bar(L::kQFull + s), 2 * L::kTileBytes);
                 for (int c = 0; c < D / 64; ++c) {
                     tma_load_3d(sbase + L::kQ + s * L::kTileBytes + c * L::kChunkBytes, &tm_q,
-                                bar(L::kQFull + s), c * 64, q0, bh);
+                                bar(L::kQFull + s), c * 64, q_y0 + q0, z);
                     tma_load_3d(sbase + L::kDO + s * L::kTileBytes + c * L::kChunkBytes, &tm_do,
-                                bar(L::kQFull + s), c * 64, q0, bh);
+                                bar(L::kQFull + s), c * 64, q_y0 + q0, z);
                 }
             }
             // row terms of this query tile: LSE in log2 units (+inf for rows
@@ -344,7 +354,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int r = lane * 4 + e;
                 const int q = q0 + r;
                 float l2 = pos_inf(), dd = 0.f;
-                if (q < p.Nq) {
+                if (q < len_q) {
                     const float l = __ldg(lse_bh + q);
                     l2 = (l == neg_inf()) ? pos_inf() : l * kLog2e;
                     dd = __ldg(di_bh + q);
@@ -468,7 +478,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int key = kv0 + row;
         const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const float qk = p.qk_scale_log2;
-        float b2 = key < p.Nk ? 0.f : neg_inf();
+        float b2 = key < len_k ? 0.f : neg_inf();
         if (HAS_BIAS && key < p.Nk)
             b2 = __ldg(p.bias + static_cast<size_t>(bh / p.H) * p.Nk + key) * kLog2e;
         // column `key` of the general mask: M[q][key] for the thread's queries
@@ -496,7 +506,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             }
             tc_fence_after();
-            const bool diag = CAUSAL && (key > qg + p.causal_off);   // some column masked
+            const bool diag = CAUSAL && (key > qg + coff);   // some column masked
             float pr[64];
             {
                 uint32_t sv[64];
@@ -522,10 +532,10 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])), qk2, c23);
                         if (!kEmu && diag) {
                             const int e = 4 * e4;
-                            if (key > qg + e + p.causal_off) x01.x = neg_inf();
-                            if (key > qg + e + 1 + p.causal_off) x01.y = neg_inf();
-                            if (key > qg + e + 2 + p.causal_off) x23.x = neg_inf();
-                            if (key > qg + e + 3 + p.causal_off) x23.y = neg_inf();
+                            if (key > qg + e + coff) x01.x = neg_inf();
+                            if (key > qg + e + 1 + coff) x01.y = neg_inf();
+                            if (key > qg + e + 2 + coff) x23.x = neg_inf();
+                            if (key > qg + e + 3 + coff) x23.y = neg_inf();
                         }
                         pr[4 * e4] = ex2_approx(x01.x);
                         pr[4 * e4 + 1] = ex2_approx(x01.y);
@@ -539,7 +549,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                 };
-                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !diag && key < p.Nk))   // warp-uniform
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !diag && key < len_k))   // warp-uniform
                     make_p(std::true_type{});
                 else
                     make_p(std::false_type{});
@@ -590,7 +600,34 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ok = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
-        if (ok) {
+        if (ok && VARLEN) {
+            // packed sequences: each thread stores its own key row (a 32-row TMA
+            // box could run into the next sequence's rows)
+            const int which = g;                            // warpgroup 0: dV, 1: dK
+            const uint32_t col = which ? L::kColDK : L::kColDV;
+            const float mul = which ? p.scale : 1.f;
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(which ? p.dk : p.dv) +
+                                                   (sr.k_row0 + key) * D);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                if (nq > 0) {
+                    tmem_ld32dp_x32_wait(tl + col + cc * 32, v);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+                if (key < len_k) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+        } else if (ok) {
             {
                 const int which = g;                        // warpgroup 0: dV, 1: dK
                 const uint32_t col = which ? L::kColDK : L::kColDV;
@@ -644,7 +681,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 //     dQ(j)      once dS(j) is over the dP columns
 //     dP(j+1)    (over dS(j), read by dQ(j) just before, in order)
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false, bool VARLEN = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -671,11 +708,18 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int qt = (n_q_all - 1) - rank_;
     const int bh = bh_;
     const int q0 = qt * kBQ;
-    const int n_kv_all = (p.Nk + kBK - 1) / kBK;
-    int n = n_kv_all;
-    if (CAUSAL) {
-        const int last_row = min(q0 + kBQ - 1, p.Nq - 1);
-        const int lim = last_row + p.causal_off;
+    // rows of this (sequence, head): fixed [B*H, N, D] layout or packed sequences
+    const SeqRows sr = VARLEN ? seq_rows(bh, p.H, p.Nq, p.Nk, p.cu_q, p.cu_k, p.total_q, p.total_k)
+                              : SeqRows{static_cast<long long>(bh) * p.Nq, static_cast<long long>(bh) * p.Nk, p.Nq, p.Nk};
+    const int len_q = sr.len_q, len_k = sr.len_k, coff = len_k - len_q;
+    const int q_y0 = VARLEN ? static_cast<int>(sr.q_row0 - static_cast<long long>(bh % p.H) * p.total_q) : 0;
+    const int k_y0 = VARLEN ? static_cast<int>(sr.k_row0 - static_cast<long long>(bh % p.H) * p.total_k) : 0;
+    const int z = VARLEN ? bh % p.H : bh;           // head slice of the tensor maps
+    const int n_kv_all = (len_k + kBK - 1) / kBK;
+    int n = q0 < len_q ? n_kv_all : 0;              // a tile past the queries: no work
+    if (CAUSAL && n > 0) {
+        const int last_row = min(q0 + kBQ - 1, len_q - 1);
+        const int lim = last_row + coff;
         n = lim < 0 ? 0 : min(n_kv_all, lim / kBK + 1);
     }
 
@@ -725,8 +769,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0 && n > 0) {
             mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTileBytes);
             for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(sbase + L::kQ + c * L::kChunkBytes, &tm_q, bar(L::kQFull), c * 64, q0, bh);
-                tma_load_3d(sbase + L::kDO + c * L::kChunkBytes, &tm_do, bar(L::kQFull), c * 64, q0, bh);
+                tma_load_3d(sbase + L::kQ + c * L::kChunkBytes, &tm_q, bar(L::kQFull), c * 64, q_y0 + q0, z);
+                tma_load_3d(sbase + L::kDO + c * L::kChunkBytes, &tm_do, bar(L::kQFull), c * 64, q_y0 + q0, z);
             }
         }
         // K runs one tile ahead of V (K_j is needed by S(j), before dP(j)).
@@ -741,7 +785,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_arrive_expect_tx(bar(L::kKFull + ks), L::kTileBytes);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sbase + L::kK + ks * L::kTileBytes + c * L::kChunkBytes, &tm_k,
-                                bar(L::kKFull + ks), c * 64, j * kBK, bh);
+                                bar(L::kKFull + ks), c * 64, k_y0 + j * kBK, z);
             }
             if constexpr (HAS_BIAS) {
                 float *bs = reinterpret_cast<float *>(smem + L::kBias) + ks * 128;
@@ -764,7 +808,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                    bar(L::kVFull + vs), c * 64, jv * kBK, bh);
+                                    bar(L::kVFull + vs), c * 64, k_y0 + jv * kBK, z);
                 }
                 v_issued = jv + 1;
             }
@@ -781,7 +825,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                    bar(L::kVFull + vs), c * 64, jv * kBK, bh);
+                                    bar(L::kVFull + vs), c * 64, k_y0 + jv * kBK, z);
                 }
                 v_issued = n;
             }
@@ -922,13 +966,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_arrive(bar(L::kQDReady));
         }
         float lse2 = pos_inf(), di = 0.f;
-        if (q < p.Nq) {
-            const float l = __ldg(p.lse + static_cast<size_t>(bh) * p.Nq + q);
+        if (q < len_q) {
+            const float l = __ldg(p.lse + sr.q_row0 + q);
             lse2 = (l == neg_inf()) ? pos_inf() : l * kLog2e;
-            di = __ldg(p.Di + static_cast<size_t>(bh) * p.Nq + q);
+            di = __ldg(p.Di + sr.q_row0 + q);
         }
         // last key this row may see
-        const int lim = CAUSAL ? min(q + p.causal_off, p.Nk - 1) : p.Nk - 1;
+        const int lim = CAUSAL ? min(q + coff, len_k - 1) : len_k - 1;
         // this row of the general mask (rows past Nq read nothing)
         const float *mrow = nullptr;
         if (HAS_MASK && q < p.Nq)
@@ -999,7 +1043,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     }
                 };
-                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !edge && q < p.Nq))   // warp-uniform
+                if (__all_sync(0xffffffffu, !HAS_BIAS && !HAS_MASK && !edge && q < len_q))   // warp-uniform
                     make_p(std::true_type{});
                 else
                     make_p(std::false_type{});
@@ -1034,7 +1078,29 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ok = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
-        if (ok) {
+        if (ok && VARLEN) {
+            // packed sequences: each thread stores its own query row
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dq) + (sr.q_row0 + q) * D);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                if (n > 0) {
+                    tmem_ld32dp_x32_wait(tl + L::kColDQ + cc * 32, v);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * p.scale, __uint_as_float(v[2 * e + 1]) * p.scale);
+                if (q < len_q) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+        } else if (ok) {
             uint8_t *stage = smem + L::kQ;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
@@ -1068,11 +1134,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false>
+template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS, bool HAS_MASK = false, bool VARLEN = false>
 cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStream_t stream) {
     {
         using L = DkdvLayout<D>;
-        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK>;
+        auto kern = fa_bwd_dkdv_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK, VARLEN>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nk + kBK - 1) / kBK) * p.B * p.H;
@@ -1084,7 +1150,7 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
     }
     {
         using L = DqLayout<D>;
-        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK>;
+        auto kern = fa_bwd_dq_kernel<D, BF16, CAUSAL, HAS_BIAS, HAS_MASK, VARLEN>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
         if (e != cudaSuccess) return e;
         const unsigned grid = static_cast<unsigned>((p.Nq + kBQ - 1) / kBQ) * p.B * p.H;
@@ -1096,10 +1162,11 @@ cudaError_t launch_grad_t(const BwdTensorMaps &tm, const BwdParams &p, cudaStrea
     }
 }
 
-// 1. D_i = rowsum(dO * O) into the workspace
+// 1. D_i = rowsum(dO * O) into the workspace (every row of the layout)
 template <int D, bool BF16>
 cudaError_t launch_pre(const BwdParams &p, cudaStream_t s) {
-    const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
+    const long long rows = p.cu_q ? static_cast<long long>(p.H) * p.total_q
+                                  : static_cast<long long>(p.B) * p.H * p.Nq;
     const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
     prof_begin(s, "fa_bwd_pre_kernel");
     fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
@@ -1115,6 +1182,14 @@ cudaError_t launch_bwd_mask_d(const BwdTensorMaps &tm, const BwdParams &p, bool 
     if (e != cudaSuccess) return e;
     return causal ? launch_grad_t<D, BF16, true, false, true>(tm, p, s)
                   : launch_grad_t<D, BF16, false, false, true>(tm, p, s);
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_varlen_d(const BwdTensorMaps &tm, const BwdParams &p, bool causal, cudaStream_t s) {
+    cudaError_t e = launch_pre<D, BF16>(p, s);
+    if (e != cudaSuccess) return e;
+    return causal ? launch_grad_t<D, BF16, true, false, false, true>(tm, p, s)
+                  : launch_grad_t<D, BF16, false, false, false, true>(tm, p, s);
 }
 
 template <int D, bool BF16>
@@ -1146,6 +1221,14 @@ cudaError_t launch_bwd_mask(const BwdTensorMaps &tm, const BwdParams &p, int D, 
                              : launch_bwd_mask_d<64, false>(tm, p, causal, stream);
     return bf16 ? launch_bwd_mask_d<128, true>(tm, p, causal, stream)
                 : launch_bwd_mask_d<128, false>(tm, p, causal, stream);
+}
+
+cudaError_t launch_bwd_varlen(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
+                              cudaStream_t stream) {
+    if (D == 64) return bf16 ? launch_bwd_varlen_d<64, true>(tm, p, causal, stream)
+                             : launch_bwd_varlen_d<64, false>(tm, p, causal, stream);
+    return bf16 ? launch_bwd_varlen_d<128, true>(tm, p, causal, stream)
+                : launch_bwd_varlen_d<128, false>(tm, p, causal, stream);
 }
 
 cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,

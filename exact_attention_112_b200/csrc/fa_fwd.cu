@@ -153,13 +153,18 @@ __device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float 
     return lo | (hi << 16);
 }
 
-// One work unit: rows [m0, m0 + 256) of head bh, key tiles
-// [kv_first, kv_first + n_kv) (n_kv == 0: the rows see no key).
+// One work unit: rows [m0, m0 + 256) of head bh (rows counted within the
+// head's sequence), key tiles [kv_first, kv_first + n_kv) (n_kv == 0: the
+// rows see no key).  The sequence has len_q queries and len_k keys; its rows
+// sit at y = q_y0 + row (k_y0 + key) of the tensor maps' head slice z, and
+// its O / LSE rows start at o_row0.
 struct Unit {
     int bh, m0, kv_first, n_kv, split;
+    int len_q, len_k, q_y0, k_y0, z;
+    long long o_row0;
 };
 
-template <bool CAUSAL, bool SPLIT>
+template <bool CAUSAL, bool SPLIT, bool VARLEN = false>
 __device__ __forceinline__ Unit unit_info(const FwdParams &p, int u) {
     Unit w;
     const int BH = p.B * p.H;
@@ -172,11 +177,27 @@ __device__ __forceinline__ Unit unit_info(const FwdParams &p, int u) {
     const int mb = (p.n_mblocks - 1) - u / BH;
     w.bh = u % BH;
     w.m0 = mb * 2 * kBM;
-    const int n_kv_all = (p.Nk + kBN - 1) / kBN;
-    w.n_kv = n_kv_all;
-    if (CAUSAL) {
-        const int last_row = min(w.m0 + 2 * kBM - 1, p.Nq - 1);
-        const int lim = last_row + p.causal_off;
+    if constexpr (VARLEN) {
+        const SeqRows sr = seq_rows(w.bh, p.H, p.Nq, p.Nk, p.cu_q, p.cu_k, p.total_q, p.total_k);
+        w.z = w.bh % p.H;
+        w.len_q = sr.len_q;
+        w.len_k = sr.len_k;
+        w.q_y0 = static_cast<int>(sr.q_row0 - static_cast<long long>(w.z) * p.total_q);
+        w.k_y0 = static_cast<int>(sr.k_row0 - static_cast<long long>(w.z) * p.total_k);
+        w.o_row0 = sr.q_row0;
+    } else {
+        w.len_q = p.Nq;
+        w.len_k = p.Nk;
+        w.q_y0 = 0;
+        w.k_y0 = 0;
+        w.z = w.bh;
+        w.o_row0 = static_cast<long long>(w.bh) * p.Nq;
+    }
+    const int n_kv_all = (w.len_k + kBN - 1) / kBN;
+    w.n_kv = w.m0 < w.len_q ? n_kv_all : 0;   // a block past the sequence's end has no rows
+    if (CAUSAL && w.n_kv > 0) {
+        const int last_row = min(w.m0 + 2 * kBM - 1, w.len_q - 1);
+        const int lim = last_row + (w.len_k - w.len_q);
         w.n_kv = lim < 0 ? 0 : min(n_kv_all, lim / kBN + 1);
     }
     w.kv_first = 0;
@@ -196,17 +217,18 @@ __device__ __forceinline__ int unit_at(const FwdParams &p, int r) {
 
 // Advance r to this CTA's next unit that has key tiles (the producer and the
 // MMA warp skip the others); false when none is left.
-template <bool CAUSAL, bool SPLIT>
+template <bool CAUSAL, bool SPLIT, bool VARLEN = false>
 __device__ __forceinline__ bool next_work(const FwdParams &p, int &r, Unit &w) {
     for (;; ++r) {
         const int u = unit_at(p, r);
         if (u < 0) return false;
-        w = unit_info<CAUSAL, SPLIT>(p, u);
+        w = unit_info<CAUSAL, SPLIT, VARLEN>(p, u);
         if (w.n_kv > 0) return true;
     }
 }
 
-template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false, bool HAS_MASK = false>
+template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS, bool SPLIT = false, bool HAS_MASK = false,
+          bool VARLEN = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -277,7 +299,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int q_issued = 0;   // Q tiles issued for the current unit
             int r = 0;
             Unit w;
-            while (ok && next_work<CAUSAL, SPLIT>(p, r, w)) {
+            while (ok && next_work<CAUSAL, SPLIT, VARLEN>(p, r, w)) {
                 // Q_i of this unit, once the previous unit's last S_i has read Q_i
                 q_issued = 0;
                 for (int i = 0; i < 2 && ok; ++i) {
@@ -285,33 +307,33 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     mbar_arrive_expect_tx(bar(L::kQFull + i), L::kTileBytes);
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kQ + i * L::kTileBytes + c * L::kChunkBytes, &tm_q,
-                                    bar(L::kQFull + i), c * L::kChunkElems, w.m0 + i * kBM, w.bh);
+                                    bar(L::kQFull + i), c * L::kChunkElems, w.q_y0 + w.m0 + i * kBM, w.z);
                     q_issued = i + 1;
                 }
                 if (!ok) break;
                 {   // warm L2 with the next unit's Q tiles
                     int r2 = r + 1;
                     Unit nx;
-                    if (next_work<CAUSAL, SPLIT>(p, r2, nx))
+                    if (next_work<CAUSAL, SPLIT, VARLEN>(p, r2, nx))
                         for (int i = 0; i < 2; ++i)
                             for (int c = 0; c < L::kChunks; ++c)
-                                tma_prefetch_l2_3d(&tm_q, c * L::kChunkElems, nx.m0 + i * kBM, nx.bh);
+                                tma_prefetch_l2_3d(&tm_q, c * L::kChunkElems, nx.q_y0 + nx.m0 + i * kBM, nx.z);
                 }
                 for (int j = 0; j < w.n_kv; ++j, ++t) {
                     const int s = t & 1;
                     const uint32_t ph = (t >> 1) & 1;
-                    const int row = (w.kv_first + j) * kBN;
+                    const int row = w.k_y0 + (w.kv_first + j) * kBN;
                     if (!mbar_wait(bar(L::kKEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kK + s * L::kTileBytes + c * L::kChunkBytes, &tm_k,
-                                    bar(L::kKFull + s), c * L::kChunkElems, row, w.bh);
+                                    bar(L::kKFull + s), c * L::kChunkElems, row, w.z);
                     ++kv_half;
                     if (!mbar_wait(bar(L::kVEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTileBytes);
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kV + s * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                    bar(L::kVFull + s), c * L::kChunkElems, row, w.bh);
+                                    bar(L::kVFull + s), c * L::kChunkElems, row, w.z);
                     ++kv_half;
                 }
                 if (!ok) break;
@@ -336,7 +358,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ============ MMA issuer (whole warp; one elected lane issues) ============
         int r = 0;
         Unit w;
-        const bool have = next_work<CAUSAL, SPLIT>(p, r, w);
+        const bool have = next_work<CAUSAL, SPLIT, VARLEN>(p, r, w);
         if (have) {
             constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32acc(kBM, kBN, false, false)
                                                : idesc_f16_f32acc(ELEM == kElemBF16, kBM, kBN, false, false);
@@ -405,7 +427,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const bool last = j + 1 == w.n_kv;
                     int r2 = r + 1;
                     Unit nx = w;
-                    const bool has_next = !last || next_work<CAUSAL, SPLIT>(p, r2, nx);
+                    const bool has_next = !last || next_work<CAUSAL, SPLIT, VARLEN>(p, r2, nx);
                     const int s1 = (t + 1) & 1;
                     const uint32_t ph1 = ((t + 1) >> 1) & 1;
                     const uint32_t pp = t & 1;
@@ -451,7 +473,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!ok) break;
                 ++uc;
                 ++r;
-                if (!next_work<CAUSAL, SPLIT>(p, r, w)) break;
+                if (!next_work<CAUSAL, SPLIT, VARLEN>(p, r, w)) break;
             }
         }
         if (have) {
@@ -483,14 +505,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int r = 0; ok; ++r) {
             const int u = unit_at(p, r);
             if (u < 0) break;
-            const Unit w = unit_info<CAUSAL, SPLIT>(p, u);
-            const int qrow = w.m0 + i * kBM + row;
+            const Unit w = unit_info<CAUSAL, SPLIT, VARLEN>(p, u);
+            const int qrow = w.m0 + i * kBM + row;   // within the head's sequence
             // last key index this row may see
-            const int lim = CAUSAL ? min(qrow + p.causal_off, p.Nk - 1) : p.Nk - 1;
+            const int lim = CAUSAL ? min(qrow + (w.len_k - w.len_q), w.len_k - 1) : w.len_k - 1;
             const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(w.bh / p.H) * p.Nk : nullptr;
             // this row of the general mask (rows past Nq read nothing)
             const float *mrow = nullptr;
-            if (HAS_MASK && qrow < p.Nq)
+            if (HAS_MASK && qrow < w.len_q)
                 mrow = p.mask + (mask_plane(w.bh, p.H, p.mask_B, p.mask_H) * p.Nq + qrow) * p.ldm;
             float m_ref = neg_inf();   // log2 units
             float l = 0.f;
@@ -670,6 +692,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (SPLIT) {
                 // partial result of this key range: O_s = o / l (fp32), LSE_s
                 const size_t prow = (static_cast<size_t>(w.split) * BH + w.bh) * p.Nq + qrow;
+                static_assert(!(SPLIT && VARLEN), "split-KV partials use the fixed layout");
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t orr[32];
@@ -690,7 +713,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (qrow < p.Nq) p.lse_part[prow] = lse;
             } else {
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) +
-                                                       (static_cast<size_t>(w.bh) * p.Nq + qrow) * D);
+                                                       (w.o_row0 + qrow) * D);
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t orr[32];
@@ -705,13 +728,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack2<kOutBF16>(__uint_as_float(orr[2 * e]) * inv_l,
                                                 __uint_as_float(orr[2 * e + 1]) * inv_l);
-                    if (qrow < p.Nq) {
+                    if (qrow < w.len_q) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4)
                             dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
                     }
                 }
-                if (qrow < p.Nq) p.lse[static_cast<size_t>(w.bh) * p.Nq + qrow] = lse;
+                if (qrow < w.len_q) p.lse[w.o_row0 + qrow] = lse;
             }
             // the next unit's first P.V may overwrite O_i only after these loads
             tc_fence_before();
@@ -801,6 +824,20 @@ cudaError_t launch_mask_t(const FwdTensorMaps &tm, const FwdParams &p, int grid,
     return cudaGetLastError();
 }
 
+template <int D, bool BF16, bool CAUSAL>
+cudaError_t launch_varlen_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
+    constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
+    using L = FwdLayout<D, kElem>;
+    auto kern = fa_fwd_kernel<D, kElem, CAUSAL, false, false, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    prof_begin(stream, "fa_fwd_varlen_kernel");
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    prof_end(stream);
+    note_launch();
+    return cudaGetLastError();
+}
+
 template <int D, bool BF16, bool CAUSAL, bool HAS_BIAS>
 cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
     constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
@@ -856,6 +893,16 @@ cudaError_t launch_fwd_mask(const FwdTensorMaps &tm, const FwdParams &p, int D, 
     }
     if (bf16) return causal ? launch_mask_t<128, true, true>(tm, p, grid, stream) : launch_mask_t<128, true, false>(tm, p, grid, stream);
     return causal ? launch_mask_t<128, false, true>(tm, p, grid, stream) : launch_mask_t<128, false, false>(tm, p, grid, stream);
+}
+
+cudaError_t launch_fwd_varlen(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                              int grid, cudaStream_t stream) {
+    if (D == 64) {
+        if (bf16) return causal ? launch_varlen_t<64, true, true>(tm, p, grid, stream) : launch_varlen_t<64, true, false>(tm, p, grid, stream);
+        return causal ? launch_varlen_t<64, false, true>(tm, p, grid, stream) : launch_varlen_t<64, false, false>(tm, p, grid, stream);
+    }
+    if (bf16) return causal ? launch_varlen_t<128, true, true>(tm, p, grid, stream) : launch_varlen_t<128, true, false>(tm, p, grid, stream);
+    return causal ? launch_varlen_t<128, false, true>(tm, p, grid, stream) : launch_varlen_t<128, false, false>(tm, p, grid, stream);
 }
 
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,

@@ -24,6 +24,12 @@ struct FwdParams {
     const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
     int mask_B, mask_H;            // 1 (broadcast) or B, H
     long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
+    // packed variable-length sequences (nullptr: fixed [B, H, N, D] layout).
+    // Then Nq, Nk are the maxima of the sequence lengths, the tensors are
+    // [H, total, D] and sequence b owns rows [cu_q[b], cu_q[b+1]) of q and o and
+    // [cu_k[b], cu_k[b+1]) of k and v.
+    const int *cu_q, *cu_k;
+    int total_q, total_k;
     void *o;                       // [B*H, Nq, D] 16-bit output
     float *lse;                    // [B*H, Nq]
     int *err;                      // device error word
@@ -49,9 +55,12 @@ struct BwdParams {
     const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
     int mask_B, mask_H;            // 1 (broadcast) or B, H
     long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
+    const int *cu_q, *cu_k;        // packed variable-length sequences (see FwdParams)
+    int total_q, total_k;
     const float *lse;              // [B*H, Nq] from the forward
     const void *o, *dO;            // [B*H, Nq, D] 16-bit
-    float *Di;                     // workspace: [B*H*Nq]
+    void *dq, *dk, *dv;            // outputs (also written through tensor maps)
+    float *Di;                     // workspace: [B*H*Nq] (packed: [H*total_q])
     int *err;
     unsigned long long timeout_ns;
 };
@@ -65,6 +74,38 @@ cudaError_t launch_bwd(const BwdTensorMaps &tm, const BwdParams &p, int D, bool 
 // Backward with the general additive mask p.mask (no key bias).
 cudaError_t launch_bwd_mask(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
                             cudaStream_t stream);
+// Backward of packed variable-length sequences (p.cu_q, p.cu_k).
+cudaError_t launch_bwd_varlen(const BwdTensorMaps &tm, const BwdParams &p, int D, bool bf16, bool causal,
+                              cudaStream_t stream);
+
+// Rows of one (sequence, head) in the packed or fixed layout: the first row
+// of its queries and keys in the [B*H or H, N or total, D] row space, and its
+// lengths.
+struct SeqRows {
+    long long q_row0, k_row0;      // first q/o row and first k/v row of (b, h)
+    int len_q, len_k;
+};
+
+__host__ __device__ inline SeqRows seq_rows(int bh, int H, int Nq, int Nk, const int *cu_q, const int *cu_k,
+                                            int total_q, int total_k) {
+    SeqRows r;
+    if (cu_q == nullptr) {
+        r.q_row0 = static_cast<long long>(bh) * Nq;
+        r.k_row0 = static_cast<long long>(bh) * Nk;
+        r.len_q = Nq;
+        r.len_k = Nk;
+    } else {
+        // the table is read as given but clamped, so that no access can leave
+        // [0, total) or exceed the maximum lengths whatever it holds
+        const int b = bh / H, h = bh % H;
+        const int q0 = min(max(cu_q[b], 0), total_q), k0 = min(max(cu_k[b], 0), total_k);
+        r.q_row0 = static_cast<long long>(h) * total_q + q0;
+        r.k_row0 = static_cast<long long>(h) * total_k + k0;
+        r.len_q = min(max(cu_q[b + 1] - q0, 0), min(Nq, total_q - q0));
+        r.len_k = min(max(cu_k[b + 1] - k0, 0), min(Nk, total_k - k0));
+    }
+    return r;
+}
 
 // Plane of the general mask used by head bh (b = bh / H, h = bh % H).
 __host__ __device__ inline long long mask_plane(int bh, int H, int mask_B, int mask_H) {
@@ -87,6 +128,9 @@ cudaError_t launch_fwd(const FwdTensorMaps &tm, const FwdParams &p, int D, int e
 // Forward with the general additive mask p.mask (16-bit inputs, no key bias).
 cudaError_t launch_fwd_mask(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                             int grid, cudaStream_t stream);
+// Forward of packed variable-length sequences (p.cu_q, p.cu_k; 16-bit inputs).
+cudaError_t launch_fwd_varlen(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
+                              int grid, cudaStream_t stream);
 cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D, bool bf16, bool causal,
                              bool has_bias, int grid, cudaStream_t stream);
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16,

@@ -168,6 +168,38 @@ int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o,
                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Forward and backward of packed variable-length sequences: num_seqs
+ * independent attention problems of different lengths stored one after
+ * another along the row axis (the "Nq != Nk / variable lengths" case; each
+ * sequence is exact attention as in fa_fwd() / fa_bwd(), with no attention
+ * across sequences).
+ *   q, o, dO, dq   [H, total_q, D];  k, v, dk, dv  [H, total_k, D];
+ *   lse            [H, total_q] float32 (same dtype and D rules as fa_fwd()).
+ *   cu_seqlens_q, cu_seqlens_k   DEVICE int32 [num_seqs + 1], non-decreasing,
+ *                  starting at 0 and ending at total_q / total_k: sequence b
+ *                  owns query rows [cu_q[b], cu_q[b+1]) and key rows
+ *                  [cu_k[b], cu_k[b+1]) of every head.
+ *   max_seqlen_q, max_seqlen_k   upper bounds of the sequence lengths (they
+ *                  size the grid; a longer sequence is cut at the bound).
+ * causal is bottom-right aligned within each sequence.  Rows of the packed
+ * tensors that belong to no sequence are not written.  The library reads the
+ * tables only on the device and clamps every start and length into [0, total]
+ * and [0, max_seqlen], so a malformed table gives wrong values, never an
+ * access outside the tensors.  The backward's workspace must hold
+ * fa_bwd_workspace_bytes(1, H, total_q, total_k, D) bytes.
+ */
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens_q, const int *cu_seqlens_k, int num_seqs, int H,
+                  int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int D,
+                  int causal, float scale, int dtype, void *stream);
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
+                  const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                  const int *cu_seqlens_q, const int *cu_seqlens_k, int num_seqs, int H,
+                  int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int D,
+                  int causal, float scale, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
+/*
  * Largest B * H * Nq that fa_bwd_noalloc() accepts.
  */
 #define FA_BWD_NOALLOC_MAX_ROWS 1048576

@@ -289,3 +289,38 @@ def test_fp8_binding_checks_types(L):
     _expect_invalid(fa.fa_fwd_fp8, "v must be torch.float8_e4m3fn",
                     q=q, k=q, v=q.to(torch.bfloat16), o=o, lse=lse)
     _expect_invalid(fa.fa_fwd_fp8, "CUDA device", q=q, k=q, v=q, o=o, lse=lse)
+
+
+def _varlen(L, cu=1, H=2, tq=100, tk=100, mq=64, mk=64, D=64, dtype=1):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    return L.fa_fwd_varlen(P(1), P(2), P(3), P(4), P(5), P(cu), P(cu), 3, H, tq, tk, mq, mk, D, 0,
+                           ctypes.c_float(0.1), dtype, None)
+
+
+def test_varlen_argument_errors_are_synchronous(L):
+    assert _varlen(L, cu=0) == fa.FA_ERR_INVALID_ARG             # no sequence table
+    assert _varlen(L, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert _varlen(L, dtype=5) == fa.FA_ERR_UNSUPPORTED
+    assert _varlen(L, tq=-1) == fa.FA_ERR_INVALID_ARG
+    assert _varlen(L, H=0) == fa.FA_ERR_INVALID_ARG
+    assert _varlen(L, mq=-1) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_fwd_varlen(*[ctypes.c_void_p(16 * i) for i in range(1, 6)], ctypes.c_void_p(18),
+                           ctypes.c_void_p(32), 3, 2, 100, 100, 64, 64, 64, 0, ctypes.c_float(0.1), 1,
+                           None) == fa.FA_ERR_INVALID_ARG        # misaligned int32 table
+    assert _varlen(L, tq=0) == fa.FA_OK                          # nothing to do, no CUDA call
+
+
+def test_varlen_binding_checks_tables(L):
+    import torch
+    q = torch.zeros((2, 10, 64), dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4, 10], dtype=torch.int32)
+    lse = torch.zeros((2, 10), dtype=torch.float32)
+    _expect_invalid(fa.fa_fwd_varlen, "cu_seqlens_q must be a contiguous int32",
+                    q=q, k=q, v=q, o=q, lse=lse, cu_seqlens_q=cu.long(), cu_seqlens_k=cu,
+                    max_seqlen_q=6, max_seqlen_k=6)
+    _expect_invalid(fa.fa_fwd_varlen, "must be on",
+                    q=q, k=q, v=q, o=q, lse=lse, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                    max_seqlen_q=6, max_seqlen_k=6)
+    _expect_invalid(fa.fa_fwd_varlen, "packed q and k must be 3-D",
+                    q=q[None], k=q, v=q, o=q, lse=lse, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                    max_seqlen_q=6, max_seqlen_k=6)
