@@ -25,7 +25,7 @@ __all__ = [
     "lib", "library_path", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes",
     "fa_bwd_noalloc",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_mask", "fa_bwd_mask",
-    "fa_fwd_varlen", "fa_bwd_varlen",
+    "fa_fwd_varlen", "fa_bwd_varlen", "fa_mask_tile_flags_bytes", "mask_tile_flags",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
     "fa_profile_enable", "fa_profile_read",
@@ -68,11 +68,15 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, vp, vp]
             L.fa_fwd_fp8.restype = i
             ll = ctypes.c_longlong
-            L.fa_fwd_mask.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, i, ll, vp]
+            L.fa_fwd_mask.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, i, ll, vp, vp]
             L.fa_fwd_mask.restype = i
             L.fa_bwd_mask.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
-                                      vp, i, i, ll, vp, sz, vp]
+                                      vp, i, i, ll, vp, vp, sz, vp]
             L.fa_bwd_mask.restype = i
+            L.fa_mask_tile_flags_bytes.argtypes = [i, i, i, i]
+            L.fa_mask_tile_flags_bytes.restype = sz
+            L.fa_mask_tile_flags.argtypes = [vp, i, i, i, i, ll, vp, sz, vp]
+            L.fa_mask_tile_flags.restype = i
             L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
             L.fa_fwd_varlen.restype = i
             L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
@@ -260,31 +264,69 @@ def _mask_args(what, mask, B, H, Nq, Nk, device):
     return Bm, Hm, ldm
 
 
-def fa_fwd_mask(q, k, v, o, lse, mask, causal=False, scale=None, stream=None):
-    """Forward with a general additive mask (see include/fa.h)."""
+def _flags_arg(what, flags, Bm, Hm, Nq, Nk, device):
+    """A mask tile summary must be a contiguous uint8 tensor of
+    fa_mask_tile_flags_bytes() elements on the mask's device (or None)."""
+    import torch
+    if flags is None:
+        return None
+    need = fa_mask_tile_flags_bytes(Bm, Hm, Nq, Nk)
+    if flags.dtype != torch.uint8 or not flags.is_contiguous() or flags.numel() != need:
+        _bad(what, f"tile_flags must be a contiguous uint8 tensor of {need} elements")
+    if not flags.is_cuda or flags.device != device:
+        _bad(what, f"tile_flags must be on {device}")
+    return flags
+
+
+def fa_mask_tile_flags_bytes(mask_B, mask_H, Nq, Nk) -> int:
+    return int(lib().fa_mask_tile_flags_bytes(mask_B, mask_H, Nq, Nk))
+
+
+def mask_tile_flags(mask, Nq=None, Nk=None, stream=None):
+    """Tile summary of a general mask (see include/fa.h, fa_mask_tile_flags):
+    a uint8 tensor [planes, ceil(Nq/128), ceil(Nk/128)], 1 where a 128 x 128
+    tile has an entry above -inf."""
+    import torch
+    m = mask if mask.dim() == 4 else mask.reshape(1, 1, *mask.shape)
+    Bm, Hm, Nq_, Nk_ = (int(x) for x in m.shape)
+    Bm, Hm, ldm = _mask_args("fa_mask_tile_flags", mask, Bm, Hm, Nq_, Nk_, mask.device)
+    out = torch.empty((Bm * Hm, (Nq_ + 127) // 128, (Nk_ + 127) // 128), dtype=torch.uint8,
+                      device=mask.device)
+    st = lib().fa_mask_tile_flags(_ptr(mask), Bm, Hm, Nq_, Nk_, ldm, _ptr(out), out.numel(),
+                                  _stream_ptr(stream))
+    _check(st, "fa_mask_tile_flags")
+    return out
+
+
+def fa_fwd_mask(q, k, v, o, lse, mask, causal=False, scale=None, tile_flags=None, stream=None):
+    """Forward with a general additive mask (see include/fa.h); tile_flags is
+    the optional summary from mask_tile_flags()."""
     B, H, Nq, Nk, D, code = _validate("fa_fwd_mask", q, k, v, o=o, lse=lse, outputs=("o", "lse"))
     Bm, Hm, ldm = _mask_args("fa_fwd_mask", mask, B, H, Nq, Nk, q.device)
+    flags = _flags_arg("fa_fwd_mask", tile_flags, Bm, Hm, Nq, Nk, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     st = lib().fa_fwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
                            int(bool(causal)), float(scale), code, _ptr(mask), Bm, Hm, ldm,
-                           _stream_ptr(stream))
+                           _ptr(flags), _stream_ptr(stream))
     _check(st, "fa_fwd_mask")
 
 
 def fa_bwd_mask(q, k, v, o, lse, dO, dq, dk, dv, workspace, mask, causal=False, scale=None,
-                stream=None):
-    """Backward with a general additive mask (see include/fa.h)."""
+                tile_flags=None, stream=None):
+    """Backward with a general additive mask (see include/fa.h); tile_flags is
+    the optional summary from mask_tile_flags()."""
     B, H, Nq, Nk, D, code = _validate("fa_bwd_mask", q, k, v, o=o, lse=lse, dO=dO, dq=dq, dk=dk,
                                       dv=dv, workspace=workspace,
                                       outputs=("o", "lse", "dO", "dq", "dk", "dv"))
     Bm, Hm, ldm = _mask_args("fa_bwd_mask", mask, B, H, Nq, Nk, q.device)
+    flags = _flags_arg("fa_bwd_mask", tile_flags, Bm, Hm, Nq, Nk, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     nbytes = workspace.numel() * workspace.element_size()
     st = lib().fa_bwd_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
                            _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, int(bool(causal)), float(scale),
-                           code, _ptr(mask), Bm, Hm, ldm, _ptr(workspace), nbytes,
+                           code, _ptr(mask), Bm, Hm, ldm, _ptr(flags), _ptr(workspace), nbytes,
                            _stream_ptr(stream))
     _check(st, "fa_bwd_mask")
 

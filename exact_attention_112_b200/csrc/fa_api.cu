@@ -214,6 +214,10 @@ fa::FwdParams fwd_params(int B, int H, int Nq, int Nk, float scale, const float 
     p.tiles_per_split = 0;
     p.cu_q = p.cu_k = nullptr;
     p.total_q = p.total_k = 0;
+    p.mask = nullptr;
+    p.mask_B = p.mask_H = 1;
+    p.ldm = 0;
+    p.tile_flags = nullptr;
     return p;
 }
 }  // namespace
@@ -303,9 +307,34 @@ int check_mask(const float *mask, int B, int H, int Nq, int Nk, int mask_B, int 
 
 extern "C" {
 
+size_t fa_mask_tile_flags_bytes(int mask_B, int mask_H, int Nq, int Nk) {
+    if (mask_B < 1 || mask_H < 1 || Nq < 0 || Nk < 0) return 0;
+    return static_cast<size_t>(mask_B) * mask_H * ((static_cast<size_t>(Nq) + 127) / 128) *
+           ((static_cast<size_t>(Nk) + 127) / 128);
+}
+
+int fa_mask_tile_flags(const float *mask, int mask_B, int mask_H, int Nq, int Nk, long long ldm,
+                       unsigned char *flags, size_t flags_bytes, void *stream) {
+    if (mask_B < 1 || mask_H < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if (mask_B > 65535 || mask_H > 65535 || static_cast<long long>(mask_B) * mask_H > 65535)
+        return FA_ERR_INVALID_ARG;   // one grid slice per plane
+    const size_t need = fa_mask_tile_flags_bytes(mask_B, mask_H, Nq, Nk);
+    if (need == 0) return FA_OK;
+    int st = check_mask(mask, mask_B, mask_H, Nq, Nk, mask_B, mask_H, ldm);
+    if (st != FA_OK) return st;
+    if (!flags || flags_bytes < need) return FA_ERR_INVALID_ARG;
+    int dev;
+    if ((st = current_device(&dev)) != FA_OK) return st;
+    int *err = nullptr;
+    if ((st = device_setup(dev, &err)) != FA_OK) return st;
+    cudaError_t e = fa::launch_mask_tile_flags(mask, mask_B * mask_H, Nq, Nk, ldm, flags,
+                                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
                 int Nq, int Nk, int D, int causal, float scale, int dtype, const float *mask,
-                int mask_B, int mask_H, long long ldm, void *stream) {
+                int mask_B, int mask_H, long long ldm, const unsigned char *tile_flags, void *stream) {
     int st = check_common(B, H, Nq, Nk, D, causal, scale, dtype);
     if (st != FA_OK) return st;
     if (Nq == 0) return FA_OK;
@@ -333,6 +362,7 @@ int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse
     p.mask_B = mask_B;
     p.mask_H = mask_H;
     p.ldm = ldm;
+    p.tile_flags = tile_flags;
     cudaError_t e = fa::launch_fwd_mask(tm, p, D, bf16, causal != 0, persistent_grid(p.n_units, sms), s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -462,7 +492,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
              const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
              int causal, float scale, int dtype, const float *key_bias, const float *mask,
              int mask_B, int mask_H, long long ldm, void *workspace, size_t workspace_bytes,
-             void *stream, const VarlenArgs &vl = VarlenArgs{}) {
+             void *stream, const VarlenArgs &vl = VarlenArgs{}, const unsigned char *tile_flags = nullptr) {
     const bool varlen = vl.cu_q != nullptr;
     int st = varlen ? check_varlen(vl.cu_q, vl.cu_k, B, H, vl.total_q, vl.total_k, Nq, Nk, D, causal, scale, dtype)
                     : check_common(B, H, Nq, Nk, D, causal, scale, dtype);
@@ -501,7 +531,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
         if (cudaMemsetAsync(dq, 0, static_cast<size_t>(q_rows) * D * 2, s) != cudaSuccess) return FA_ERR_CUDA;
         return FA_OK;
     }
-    fa::BwdParams p;
+    fa::BwdParams p{};
     p.B = B;
     p.H = H;
     p.Nq = Nq;
@@ -514,6 +544,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     p.mask_B = mask_B;
     p.mask_H = mask_H;
     p.ldm = ldm;
+    p.tile_flags = mask ? tile_flags : nullptr;
     p.lse = lse;
     p.o = o;
     p.dO = dO;
@@ -575,10 +606,11 @@ int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, co
 int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o, const float *lse,
                 const void *dO, void *dq, void *dk, void *dv, int B, int H, int Nq, int Nk, int D,
                 int causal, float scale, int dtype, const float *mask, int mask_B, int mask_H,
-                long long ldm, void *workspace, size_t workspace_bytes, void *stream) {
+                long long ldm, const unsigned char *tile_flags, void *workspace, size_t workspace_bytes,
+                void *stream) {
     if (!mask) return FA_ERR_INVALID_ARG;
     return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, causal, scale, dtype, nullptr,
-                    mask, mask_B, mask_H, ldm, workspace, workspace_bytes, stream);
+                    mask, mask_B, mask_H, ldm, workspace, workspace_bytes, stream, VarlenArgs{}, tile_flags);
 }
 
 int fa_device_status(void *stream) {

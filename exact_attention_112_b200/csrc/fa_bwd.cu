@@ -177,6 +177,34 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
     }
 }
 
+// With a general mask and its tile summary, the recompute kernels visit only
+// the tiles the summary marks: the first query tile q >= from (of key tile
+// kt) and the first key tile k >= from (of query tile qt) that must be visited,
+// or `end` if none.  Without one, every tile in the range is visited.
+template <bool HAS_MASK>
+__device__ __forceinline__ int next_qtile(const BwdParams &p, long long plane, int kt, int from, int end) {
+    if constexpr (HAS_MASK) {
+        if (p.tile_flags != nullptr) {
+            for (int q = from; q < end; ++q)
+                if (mask_tile_needed(p.tile_flags, plane, p.Nq, p.Nk, q, kt)) return q;
+            return end;
+        }
+    }
+    return from;
+}
+
+template <bool HAS_MASK>
+__device__ __forceinline__ int next_ktile(const BwdParams &p, long long plane, int qt, int from, int end) {
+    if constexpr (HAS_MASK) {
+        if (p.tile_flags != nullptr) {
+            for (int k = from; k < end; ++k)
+                if (mask_tile_needed(p.tile_flags, plane, p.Nq, p.Nk, qt, k)) return k;
+            return end;
+        }
+    }
+    return from;
+}
+
 // ---------------------------------------------------------------------------
 // 1. D_i = rowsum(dO * O).  One warp per row.
 // ---------------------------------------------------------------------------
@@ -281,7 +309,14 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         j_begin = first_q > 0 ? first_q / kBQ : 0;
         if (j_begin > n_q_all) j_begin = n_q_all;
     }
-    const int nq = n_q_all - j_begin;
+    const long long plane = HAS_MASK ? mask_plane(bh, p.H, p.mask_B, p.mask_H) : 0;
+    int nq = n_q_all - j_begin;      // query tiles this key tile visits
+    if (HAS_MASK && p.tile_flags != nullptr) {
+        nq = 0;
+        for (int q = next_qtile<HAS_MASK>(p, plane, t, j_begin, n_q_all); q < n_q_all;
+             q = next_qtile<HAS_MASK>(p, plane, t, q + 1, n_q_all))
+            ++nq;
+    }
 
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -330,10 +365,11 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tma_load_3d(sbase + L::kV + c * L::kChunkBytes, &tm_v, bar(L::kKVFull), c * 64, k_y0 + kv0, z);
             }
         }
-        for (int jj = 0; jj < nq; ++jj) {
+        int qt = next_qtile<HAS_MASK>(p, plane, t, j_begin, n_q_all);   // query tile of step jj
+        for (int jj = 0; jj < nq; ++jj, qt = next_qtile<HAS_MASK>(p, plane, t, qt + 1, n_q_all)) {
             const int s = jj & 1;
             const uint32_t ph = (jj >> 1) & 1;
-            const int q0 = (j_begin + jj) * kBQ;
+            const int q0 = qt * kBQ;
             const bool got = mbar_wait(bar(L::kQEmpty + s), ph ^ 1, wctx);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             if (lane == 0) {
@@ -485,11 +521,12 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // (consecutive keys across the warp, so every load is one 128-byte line)
         const float *mcol = nullptr;
         if (HAS_MASK && key < p.Nk)
-            mcol = p.mask + mask_plane(bh, p.H, p.mask_B, p.mask_H) * p.Nq * p.ldm + key;
+            mcol = p.mask + plane * p.Nq * p.ldm + key;
         bool ok = true;
-        for (int jj = 0; jj < nq; ++jj) {
+        int qt = next_qtile<HAS_MASK>(p, plane, t, j_begin, n_q_all);   // query tile of step jj
+        for (int jj = 0; jj < nq; ++jj, qt = next_qtile<HAS_MASK>(p, plane, t, qt + 1, n_q_all)) {
             const int s = jj & 1;
-            const int qg = (j_begin + jj) * kBQ + 64 * g;     // first query of this thread's half
+            const int qg = qt * kBQ + 64 * g;                 // first query of this thread's half
             const float *rowbuf = reinterpret_cast<const float *>(smem + L::kRow) + s * 256 + 64 * g;
             float mk[HAS_MASK ? 64 : 1];
             if constexpr (HAS_MASK) {
@@ -722,6 +759,14 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int lim = last_row + coff;
         n = lim < 0 ? 0 : min(n_kv_all, lim / kBK + 1);
     }
+    const int n_range = n;                          // key tiles [0, n_range) may be visible
+    const long long plane = HAS_MASK ? mask_plane(bh, p.H, p.mask_B, p.mask_H) : 0;
+    if (HAS_MASK && p.tile_flags != nullptr) {     // visit only the tiles the summary marks
+        n = 0;
+        for (int k = next_ktile<HAS_MASK>(p, plane, qt, 0, n_range); k < n_range;
+             k = next_ktile<HAS_MASK>(p, plane, qt, k + 1, n_range))
+            ++n;
+    }
 
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -774,7 +819,8 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         // K runs one tile ahead of V (K_j is needed by S(j), before dP(j)).
-        for (int j = 0; j < n && ok; ++j) {
+        int kt = next_ktile<HAS_MASK>(p, plane, qt, 0, n_range), kt_prev = -1;   // key tiles of steps j, j-1
+        for (int j = 0; j < n && ok; ++j, kt_prev = kt, kt = next_ktile<HAS_MASK>(p, plane, qt, kt + 1, n_range)) {
             const int ks = j % L::kKStages;
             const uint32_t kph = (j / L::kKStages) & 1;
             {
@@ -785,13 +831,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_arrive_expect_tx(bar(L::kKFull + ks), L::kTileBytes);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sbase + L::kK + ks * L::kTileBytes + c * L::kChunkBytes, &tm_k,
-                                bar(L::kKFull + ks), c * 64, k_y0 + j * kBK, z);
+                                bar(L::kKFull + ks), c * 64, k_y0 + kt * kBK, z);
             }
             if constexpr (HAS_BIAS) {
                 float *bs = reinterpret_cast<float *>(smem + L::kBias) + ks * 128;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int key = j * kBK + lane * 4 + e;
+                    const int key = kt * kBK + lane * 4 + e;
                     bs[lane * 4 + e] = key < p.Nk ? __ldg(bias_b + key) * kLog2e : neg_inf();
                 }
                 __syncwarp();
@@ -808,7 +854,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                    bar(L::kVFull + vs), c * 64, k_y0 + jv * kBK, z);
+                                    bar(L::kVFull + vs), c * 64, k_y0 + kt_prev * kBK, z);
                 }
                 v_issued = jv + 1;
             }
@@ -825,7 +871,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mbar_arrive_expect_tx(bar(L::kVFull + vs), L::kTileBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + L::kV + vs * L::kTileBytes + c * L::kChunkBytes, &tm_v,
-                                    bar(L::kVFull + vs), c * 64, k_y0 + jv * kBK, z);
+                                    bar(L::kVFull + vs), c * 64, k_y0 + kt_prev * kBK, z);
                 }
                 v_issued = n;
             }
@@ -976,9 +1022,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // this row of the general mask (rows past Nq read nothing)
         const float *mrow = nullptr;
         if (HAS_MASK && q < p.Nq)
-            mrow = p.mask + (mask_plane(bh, p.H, p.mask_B, p.mask_H) * p.Nq + q) * p.ldm;
-        for (int j = 0; j < n && ok; ++j) {
-            const int kg = j * kBK + 64 * g;                  // first key of this thread's half
+            mrow = p.mask + (plane * p.Nq + q) * p.ldm;
+        int kt = next_ktile<HAS_MASK>(p, plane, qt, 0, n_range);   // key tile of step j
+        for (int j = 0; j < n && ok; ++j, kt = next_ktile<HAS_MASK>(p, plane, qt, kt + 1, n_range)) {
+            const int kg = kt * kBK + 64 * g;                 // first key of this thread's half
             float mk[HAS_MASK ? 64 : 1];
             if constexpr (HAS_MASK) {
                 // issued before the wait for S so the loads overlap it

@@ -162,9 +162,30 @@ struct Unit {
     int bh, m0, kv_first, n_kv, split;
     int len_q, len_k, q_y0, k_y0, z;
     long long o_row0;
+    // with a general mask and its tile summary, the unit visits only the key
+    // tiles in [kv_first, kv_end) that the summary marks for one of its two
+    // query tiles; n_kv counts those
+    int kv_end;
+    long long plane;
 };
 
-template <bool CAUSAL, bool SPLIT, bool VARLEN = false>
+// First key tile k >= from of the unit that must be visited (kv_end if none).
+template <bool HAS_MASK>
+__device__ __forceinline__ int next_tile(const FwdParams &p, const Unit &w, int from) {
+    if constexpr (HAS_MASK) {
+        if (p.tile_flags != nullptr) {
+            const int qt0 = w.m0 / kBM;
+            for (int k = from; k < w.kv_end; ++k)
+                if (mask_tile_needed(p.tile_flags, w.plane, p.Nq, p.Nk, qt0, k) ||
+                    mask_tile_needed(p.tile_flags, w.plane, p.Nq, p.Nk, qt0 + 1, k))
+                    return k;
+            return w.kv_end;
+        }
+    }
+    return from;
+}
+
+template <bool CAUSAL, bool SPLIT, bool VARLEN = false, bool HAS_MASK = false>
 __device__ __forceinline__ Unit unit_info(const FwdParams &p, int u) {
     Unit w;
     const int BH = p.B * p.H;
@@ -205,6 +226,16 @@ __device__ __forceinline__ Unit unit_info(const FwdParams &p, int u) {
         w.kv_first = w.split * p.tiles_per_split;
         w.n_kv = max(0, min(w.n_kv, w.kv_first + p.tiles_per_split) - w.kv_first);
     }
+    w.kv_end = w.kv_first + w.n_kv;
+    w.plane = 0;
+    if constexpr (HAS_MASK) {
+        w.plane = mask_plane(w.bh, p.H, p.mask_B, p.mask_H);
+        if (p.tile_flags != nullptr) {
+            int n = 0;
+            for (int k = next_tile<true>(p, w, w.kv_first); k < w.kv_end; k = next_tile<true>(p, w, k + 1)) ++n;
+            w.n_kv = n;
+        }
+    }
     return w;
 }
 
@@ -217,12 +248,12 @@ __device__ __forceinline__ int unit_at(const FwdParams &p, int r) {
 
 // Advance r to this CTA's next unit that has key tiles (the producer and the
 // MMA warp skip the others); false when none is left.
-template <bool CAUSAL, bool SPLIT, bool VARLEN = false>
+template <bool CAUSAL, bool SPLIT, bool VARLEN = false, bool HAS_MASK = false>
 __device__ __forceinline__ bool next_work(const FwdParams &p, int &r, Unit &w) {
     for (;; ++r) {
         const int u = unit_at(p, r);
         if (u < 0) return false;
-        w = unit_info<CAUSAL, SPLIT, VARLEN>(p, u);
+        w = unit_info<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, u);
         if (w.n_kv > 0) return true;
     }
 }
@@ -299,7 +330,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int q_issued = 0;   // Q tiles issued for the current unit
             int r = 0;
             Unit w;
-            while (ok && next_work<CAUSAL, SPLIT, VARLEN>(p, r, w)) {
+            while (ok && next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r, w)) {
                 // Q_i of this unit, once the previous unit's last S_i has read Q_i
                 q_issued = 0;
                 for (int i = 0; i < 2 && ok; ++i) {
@@ -314,15 +345,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 {   // warm L2 with the next unit's Q tiles
                     int r2 = r + 1;
                     Unit nx;
-                    if (next_work<CAUSAL, SPLIT, VARLEN>(p, r2, nx))
+                    if (next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r2, nx))
                         for (int i = 0; i < 2; ++i)
                             for (int c = 0; c < L::kChunks; ++c)
                                 tma_prefetch_l2_3d(&tm_q, c * L::kChunkElems, nx.q_y0 + nx.m0 + i * kBM, nx.z);
                 }
-                for (int j = 0; j < w.n_kv; ++j, ++t) {
+                int kt = next_tile<HAS_MASK>(p, w, w.kv_first);      // key tile of step j
+                for (int j = 0; j < w.n_kv; ++j, ++t, kt = next_tile<HAS_MASK>(p, w, kt + 1)) {
                     const int s = t & 1;
                     const uint32_t ph = (t >> 1) & 1;
-                    const int row = w.k_y0 + (w.kv_first + j) * kBN;
+                    const int row = w.k_y0 + kt * kBN;
                     if (!mbar_wait(bar(L::kKEmpty + s), ph ^ 1, wctx)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTileBytes);
                     for (int c = 0; c < L::kChunks; ++c)
@@ -358,7 +390,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ============ MMA issuer (whole warp; one elected lane issues) ============
         int r = 0;
         Unit w;
-        const bool have = next_work<CAUSAL, SPLIT, VARLEN>(p, r, w);
+        const bool have = next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r, w);
         if (have) {
             constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32acc(kBM, kBN, false, false)
                                                : idesc_f16_f32acc(ELEM == kElemBF16, kBM, kBN, false, false);
@@ -427,7 +459,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const bool last = j + 1 == w.n_kv;
                     int r2 = r + 1;
                     Unit nx = w;
-                    const bool has_next = !last || next_work<CAUSAL, SPLIT, VARLEN>(p, r2, nx);
+                    const bool has_next = !last || next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r2, nx);
                     const int s1 = (t + 1) & 1;
                     const uint32_t ph1 = ((t + 1) >> 1) & 1;
                     const uint32_t pp = t & 1;
@@ -473,7 +505,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!ok) break;
                 ++uc;
                 ++r;
-                if (!next_work<CAUSAL, SPLIT, VARLEN>(p, r, w)) break;
+                if (!next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r, w)) break;
             }
         }
         if (have) {
@@ -505,7 +537,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int r = 0; ok; ++r) {
             const int u = unit_at(p, r);
             if (u < 0) break;
-            const Unit w = unit_info<CAUSAL, SPLIT, VARLEN>(p, u);
+            const Unit w = unit_info<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, u);
             const int qrow = w.m0 + i * kBM + row;   // within the head's sequence
             // last key index this row may see
             const int lim = CAUSAL ? min(qrow + (w.len_k - w.len_q), w.len_k - 1) : w.len_k - 1;
@@ -516,8 +548,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mrow = p.mask + (mask_plane(w.bh, p.H, p.mask_B, p.mask_H) * p.Nq + qrow) * p.ldm;
             float m_ref = neg_inf();   // log2 units
             float l = 0.f;
-            for (int j = 0; j < w.n_kv; ++j, ++t) {
-                const int kv0 = (w.kv_first + j) * kBN;
+            int kt = next_tile<HAS_MASK>(p, w, w.kv_first);          // key tile of step j
+            for (int j = 0; j < w.n_kv; ++j, ++t, kt = next_tile<HAS_MASK>(p, w, kt + 1)) {
+                const int kv0 = kt * kBN;
                 {
                     const bool got = mbar_wait(bar(L::kSFull + i), t & 1, wctx);
                     if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -787,6 +820,33 @@ __global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const float *__rest
     }
 }
 
+// Tile summary of a general mask: flags[plane][qt][kt] = 1 if any entry of the
+// 128 x 128 tile (query rows qt*128.., keys kt*128..) is above -inf.  One
+// block per tile; each warp reads whole 128-value row segments (coalesced).
+__global__ void __launch_bounds__(128) fa_mask_flags_kernel(const float *__restrict__ mask, int Nq, int Nk,
+                                                            long long ldm, uint8_t *__restrict__ flags) {
+    const int kt = blockIdx.x, qt = blockIdx.y;
+    const long long plane = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int k0 = kt * 128 + lane * 4;
+    bool any = false;
+    for (int r = warp; r < 128; r += 4) {
+        const int q = qt * 128 + r;
+        if (q >= Nq) break;
+        const float *row = mask + (plane * Nq + q) * ldm;
+        if (k0 + 3 < Nk) {
+            const float4 m = __ldg(reinterpret_cast<const float4 *>(row + k0));
+            any |= m.x > neg_inf() || m.y > neg_inf() || m.z > neg_inf() || m.w > neg_inf();
+        } else {
+            for (int e = 0; e < 4; ++e)
+                if (k0 + e < Nk) any |= __ldg(row + k0 + e) > neg_inf();
+        }
+    }
+    const int hit = __syncthreads_or(any ? 1 : 0);
+    if (threadIdx.x == 0)
+        flags[(plane * gridDim.y + qt) * gridDim.x + kt] = hit ? 1 : 0;
+}
+
 // Rows with no key at all (Nk == 0): O = 0, LSE = -inf.
 template <typename T>
 __global__ void fa_fwd_empty_kernel(T *o, float *lse, size_t n_rows, int D) {
@@ -911,6 +971,17 @@ cudaError_t launch_fwd_split(const FwdTensorMaps &tm, const FwdParams &p, int D,
                              : launch_split_d<64, false>(tm, p, causal, has_bias, grid, stream);
     return bf16 ? launch_split_d<128, true>(tm, p, causal, has_bias, grid, stream)
                 : launch_split_d<128, false>(tm, p, causal, has_bias, grid, stream);
+}
+
+cudaError_t launch_mask_tile_flags(const float *mask, int planes, int Nq, int Nk, long long ldm, uint8_t *flags,
+                                   cudaStream_t stream) {
+    const dim3 grid((Nk + 127) / 128, (Nq + 127) / 128, planes);
+    if (grid.x == 0 || grid.y == 0) return cudaSuccess;
+    prof_begin(stream, "fa_mask_flags_kernel");
+    fa_mask_flags_kernel<<<grid, 128, 0, stream>>>(mask, Nq, Nk, ldm, flags);
+    prof_end(stream);
+    note_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_empty(void *o, float *lse, size_t n_rows, int D, bool bf16, cudaStream_t stream) {

@@ -24,6 +24,7 @@ struct FwdParams {
     const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
     int mask_B, mask_H;            // 1 (broadcast) or B, H
     long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
+    const uint8_t *tile_flags;     // [mask planes, ceil(Nq/128), ceil(Nk/128)] or nullptr
     // packed variable-length sequences (nullptr: fixed [B, H, N, D] layout).
     // Then Nq, Nk are the maxima of the sequence lengths, the tensors are
     // [H, total, D] and sequence b owns rows [cu_q[b], cu_q[b+1]) of q and o and
@@ -55,6 +56,7 @@ struct BwdParams {
     const float *mask;             // [mask_B, mask_H, Nq, ldm] or nullptr
     int mask_B, mask_H;            // 1 (broadcast) or B, H
     long long ldm;                 // mask row stride (elements, multiple of 4, >= Nk)
+    const uint8_t *tile_flags;     // [mask planes, ceil(Nq/128), ceil(Nk/128)] or nullptr
     const int *cu_q, *cu_k;        // packed variable-length sequences (see FwdParams)
     int total_q, total_k;
     const float *lse;              // [B*H, Nq] from the forward
@@ -105,6 +107,21 @@ __host__ __device__ inline SeqRows seq_rows(int bh, int H, int Nq, int Nk, const
         r.len_k = min(max(cu_k[b + 1] - k0, 0), min(Nk, total_k - k0));
     }
     return r;
+}
+
+// Summary of a general mask: one byte per 128 x 128 tile of each plane, 1 if
+// any entry of the tile is above -inf (fa_mask_tile_flags).
+cudaError_t launch_mask_tile_flags(const float *mask, int planes, int Nq, int Nk, long long ldm,
+                                   uint8_t *flags, cudaStream_t stream);
+
+// Does the 128-row query tile qt of mask plane `plane` need key tile kt?
+// (Without a summary every tile is needed.)
+__host__ __device__ inline bool mask_tile_needed(const uint8_t *flags, long long plane, int Nq, int Nk, int qt,
+                                                 int kt) {
+    if (flags == nullptr) return true;
+    const int n_qt = (Nq + 127) / 128, n_kt = (Nk + 127) / 128;
+    if (qt < 0 || qt >= n_qt) return false;
+    return flags[(plane * n_qt + qt) * n_kt + kt] != 0;
 }
 
 // Plane of the general mask used by head bh (b = bh / H, h = bh % H).

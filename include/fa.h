@@ -157,15 +157,28 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
  * of fa_fwd() and fa_bwd(); the mask adds Nq * Nk * 4 bytes of reads per
  * plane, so these calls are bound by memory bandwidth rather than the tensor
  * cores.  Invalid mask arguments return FA_ERR_INVALID_ARG.
+ *
+ * tile_flags (optional, NULL = visit every tile) is the mask's tile summary
+ * written by fa_mask_tile_flags() for the same mask and sizes: device bytes
+ * [mask_B * mask_H, ceil(Nq/128), ceil(Nk/128)], 1 where a 128 x 128 tile
+ * has an entry above -inf.  Tiles marked 0 contribute exactly nothing and are
+ * skipped (not loaded, not multiplied), so masks that hide whole blocks --
+ * packed documents, sliding windows -- cost only their visible tiles.  One
+ * summary serves the forward and the backward and every call with that mask.
  */
+size_t fa_mask_tile_flags_bytes(int mask_B, int mask_H, int Nq, int Nk);
+int fa_mask_tile_flags(const float *mask, int mask_B, int mask_H, int Nq, int Nk,
+                       long long ldm, unsigned char *flags, size_t flags_bytes, void *stream);
 int fa_fwd_mask(const void *q, const void *k, const void *v, void *o, float *lse,
                 int B, int H, int Nq, int Nk, int D, int causal, float scale, int dtype,
-                const float *mask, int mask_B, int mask_H, long long ldm, void *stream);
+                const float *mask, int mask_B, int mask_H, long long ldm,
+                const unsigned char *tile_flags, void *stream);
 int fa_bwd_mask(const void *q, const void *k, const void *v, const void *o,
                 const float *lse, const void *dO, void *dq, void *dk, void *dv,
                 int B, int H, int Nq, int Nk, int D, int causal, float scale,
                 int dtype, const float *mask, int mask_B, int mask_H, long long ldm,
-                void *workspace, size_t workspace_bytes, void *stream);
+                const unsigned char *tile_flags, void *workspace, size_t workspace_bytes,
+                void *stream);
 
 /*
  * Forward and backward of packed variable-length sequences: num_seqs

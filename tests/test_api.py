@@ -324,3 +324,18 @@ def test_varlen_binding_checks_tables(L):
     _expect_invalid(fa.fa_fwd_varlen, "packed q and k must be 3-D",
                     q=q[None], k=q, v=q, o=q, lse=lse, cu_seqlens_q=cu, cu_seqlens_k=cu,
                     max_seqlen_q=6, max_seqlen_k=6)
+
+
+def test_mask_tile_flags_arguments(L):
+    P = lambda x: None if x is None else ctypes.c_void_p(16 * x if x else 0)
+    assert fa.fa_mask_tile_flags_bytes(2, 3, 300, 129) == 2 * 3 * 3 * 2
+    assert fa.fa_mask_tile_flags_bytes(0, 1, 10, 10) == 0
+    call = lambda mask=1, Bm=1, Hm=1, Nq=300, Nk=200, ldm=200, flags=2, nbytes=1 << 20: \
+        L.fa_mask_tile_flags(P(mask), Bm, Hm, Nq, Nk, ldm, P(flags), nbytes, None)
+    assert call(mask=0) == fa.FA_ERR_INVALID_ARG
+    assert call(ldm=198) == fa.FA_ERR_INVALID_ARG          # not a multiple of 4
+    assert call(ldm=196) == fa.FA_ERR_INVALID_ARG          # shorter than Nk
+    assert call(flags=0) == fa.FA_ERR_INVALID_ARG
+    assert call(nbytes=5) == fa.FA_ERR_INVALID_ARG         # 3 x 2 tiles need 6 bytes
+    assert call(Bm=0) == fa.FA_ERR_INVALID_ARG
+    assert call(Nq=0, mask=None, flags=None) == fa.FA_OK   # no tile: nothing to do

@@ -24,7 +24,8 @@ from gpu_util import TOL_GRAD_REL, compare_fwd, compare_grads
 pytestmark = pytest.mark.gpu
 
 
-def _case(B, H, Nq, Nk, D, dtype, causal, kind, planes, seed, ldm=None, backward=True, rows=None):
+def _case(B, H, Nq, Nk, D, dtype, causal, kind, planes, seed, ldm=None, backward=True, rows=None,
+          use_flags=False):
     inp = inputs.make_inputs(B, H, Nq, Nk, D, dtype=dtype, seed=seed, with_dO=backward)
     Bm = B if planes[0] else 1
     Hm = H if planes[1] else 1
@@ -35,7 +36,8 @@ def _case(B, H, Nq, Nk, D, dtype, causal, kind, planes, seed, ldm=None, backward
     mdev = mbuf.to(dev)[..., :Nk]
     o = torch.full_like(q, float("nan"))
     lse = torch.full((B, H, Nq), float("nan"), dtype=torch.float32, device=dev)
-    fa.fa_fwd_mask(q, k, v, o, lse, mdev, causal=causal)
+    flags = fa.mask_tile_flags(mdev) if use_flags else None
+    fa.fa_fwd_mask(q, k, v, o, lse, mdev, causal=causal, tile_flags=flags)
     torch.cuda.synchronize()
     assert fa.fa_device_status() == fa.FA_OK
     f = inputs.to_f64
@@ -54,7 +56,7 @@ def _case(B, H, Nq, Nk, D, dtype, causal, kind, planes, seed, ldm=None, backward
     dk = torch.full_like(k, float("nan"))
     dv = torch.full_like(v, float("nan"))
     ws = torch.full((fa.fa_bwd_workspace_bytes(B, H, Nq, Nk, D),), 0xFF, dtype=torch.uint8, device=dev)
-    fa.fa_bwd_mask(q, k, v, o, lse, do, dq, dk, dv, ws, mdev, causal=causal)
+    fa.fa_bwd_mask(q, k, v, o, lse, do, dq, dk, dv, ws, mdev, causal=causal, tile_flags=flags)
     torch.cuda.synchronize()
     assert fa.fa_device_status() == fa.FA_OK
     ref = oracle.bwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["do"]), None, causal, scale,
@@ -122,3 +124,45 @@ def test_zero_mask_equals_plain_attention():
     # the scores on the FMA pipe; the mask path uses MUFU throughout)
     assert float((o1.float() - o2.float()).abs().max()) <= 2e-2
     assert float((l1 - l2).abs().max()) <= 1e-3
+
+
+def _host_flags(mask):
+    """The tile summary recomputed on the host: 1 where a 128 x 128 tile of a
+    plane has an entry above -inf."""
+    m = mask.detach().cpu().double().numpy()
+    if m.ndim == 2:
+        m = m[None, None]
+    P = m.shape[0] * m.shape[1]
+    m = m.reshape(P, m.shape[2], m.shape[3])
+    nq, nk = -(-m.shape[1] // 128), -(-m.shape[2] // 128)
+    out = np.zeros((P, nq, nk), dtype=np.uint8)
+    for pl in range(P):
+        for a in range(nq):
+            for b in range(nk):
+                out[pl, a, b] = np.any(m[pl, a * 128:(a + 1) * 128, b * 128:(b + 1) * 128] > -np.inf)
+    return out
+
+
+@pytest.mark.parametrize("kind,planes", [("document", (1, 1)), ("window", (2, 1)), ("random", (1, 3)),
+                                         ("rows", (2, 2))])
+def test_tile_flags_match_the_mask(kind, planes):
+    m = inputs.make_mask(kind, 700, 900, seed=21, planes=planes)
+    mdev = (m._base if m._base is not None else m).cuda()[..., :900]
+    flags = fa.mask_tile_flags(mdev)
+    torch.cuda.synchronize()
+    assert np.array_equal(flags.cpu().numpy(), _host_flags(m))
+
+
+@pytest.mark.parametrize("kind", ["document", "window", "rows"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tile_skipping_parity(kind, causal):
+    # with the summary, tiles that are entirely -inf are skipped; results as the oracle
+    _case(1, 2, 1100, 1100, 64, "bf16", causal, kind, (False, False), seed=22, use_flags=True)
+    _case(2, 2, 700, 900, 128, "f16", False, kind, (True, False), seed=23, use_flags=True)
+
+
+def test_tile_skipping_long_document_mask():
+    N = 4096
+    rows = inputs.sample_rows(N, seed=4)
+    _case(1, 4, N, N, 128, "bf16", False, "document", (False, False), seed=24, backward=False,
+          rows=rows, use_flags=True)
