@@ -123,12 +123,17 @@ struct FwdLayout {
     static constexpr int kDrain = 20;
     static constexpr int kNumBars = 21;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
-    static constexpr int kBytes = kMisc + 16;
+    // per softmax warp: two slots of one key tile of bias (fp32)
+    static constexpr int kBiasStage = (kMisc + 16 + 15) / 16 * 16;
+    static constexpr int kBiasSlot = kBN * 4;
+    static constexpr int kBytes = kBiasStage + 8 * 2 * kBiasSlot;
     static constexpr int kAlloc = kBytes + 1024;       // room to align the base
+    static constexpr int kAllocNoBias = kBiasStage + 1024;   // kernels without a key bias
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
     static_assert(kChunks >= 1 && kRowBytes % 128 == 0, "rows must be whole 128-byte swizzle rows");
     static_assert(kAlloc <= 232448, "shared memory");
+    static_assert(kBiasStage % 16 == 0, "float4 bias slots");
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -531,6 +536,26 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t tS = tl + (i ? L::kColS1 : L::kColS0);
         const uint32_t tO = tl + (i ? L::kColO1 : L::kColO0);
         const float qk = p.qk_scale_log2;
+        // Key bias: every row of a tile adds the same 128 values.  Each warp
+        // copies them (cp.async, four per lane) into its own shared-memory slot
+        // one tile ahead, scales them by log2(e) in place when the tile starts,
+        // and the tile reads them as broadcasts.  Two slots alternate by tile.
+        uint8_t *bslots = smem + L::kBiasStage + warp * 2 * L::kBiasSlot;
+        auto bias_fetch = [&](const float *bias_b, int kv0, int slot) {
+            const int c0 = kv0 + 4 * lane;
+            const float *src = bias_b + c0;
+            const uint32_t dst = smem_u32(bslots + slot * L::kBiasSlot + 16 * lane);
+            if ((reinterpret_cast<uintptr_t>(bias_b) & 15) == 0 && (p.Nk & 3) == 0) {
+                const int n = min(max(p.Nk - c0, 0), 4);
+                cp_async_zfill<16>(dst, n > 0 ? src : bias_b, 4 * n);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool in = c0 + e < p.Nk;
+                    cp_async_zfill<4>(dst + 4 * e, in ? src + e : bias_b, in ? 4 : 0);
+                }
+            }
+        };
         bool ok = true;
         int t = 0;      // key tiles seen so far (S/P barrier phases)
         int uc = 0;     // units with key tiles done so far (O barrier phase)
@@ -542,6 +567,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // last key index this row may see
             const int lim = CAUSAL ? min(qrow + (w.len_k - w.len_q), w.len_k - 1) : w.len_k - 1;
             const float *bias_b = HAS_BIAS ? p.bias + static_cast<size_t>(w.bh / p.H) * p.Nk : nullptr;
+            if constexpr (HAS_BIAS) {
+                if (w.n_kv > 0) bias_fetch(bias_b, next_tile<HAS_MASK>(p, w, w.kv_first) * kBN, t & 1);
+                cp_async_commit();
+            }
             // this row of the general mask (rows past Nq read nothing)
             const float *mrow = nullptr;
             if (HAS_MASK && qrow < w.len_q)
@@ -551,6 +580,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int kt = next_tile<HAS_MASK>(p, w, w.kv_first);          // key tile of step j
             for (int j = 0; j < w.n_kv; ++j, ++t, kt = next_tile<HAS_MASK>(p, w, kt + 1)) {
                 const int kv0 = kt * kBN;
+                if constexpr (HAS_BIAS) {
+                    // every lane has finished reading the other slot (previous
+                    // tile) before it is refilled with the next tile's bias
+                    __syncwarp();
+                    if (j + 1 < w.n_kv) bias_fetch(bias_b, next_tile<HAS_MASK>(p, w, kt + 1) * kBN, (t + 1) & 1);
+                    cp_async_commit();
+                    cp_async_wait<1>();          // this tile's copy has landed
+                    float4 *mine = reinterpret_cast<float4 *>(bslots + (t & 1) * L::kBiasSlot) + lane;
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    const float4 b = *mine;
+                    *mine = make_float4(b.x * kLog2e, b.y * kLog2e, b.z * kLog2e, b.w * kLog2e);
+                    __syncwarp();
+                }
                 {
                     const bool got = mbar_wait(bar(L::kSFull + i), t & 1, wctx);
                     if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -560,26 +602,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_ld32dp_x128_wait(tS, sr);
                 float x[128];
                 if constexpr (HAS_BIAS) {
-                    // x = s * qk_scale + bias * log2(e); every lane reads the same
-                    // addresses, so each load is one broadcast transaction.
-                    constexpr float kLog2e = 1.4426950408889634f;
-                    const float *bt = bias_b + kv0;
-                    if (kv0 + kBN <= p.Nk && (reinterpret_cast<uintptr_t>(bt) & 15) == 0) {
-                        const float4 *b4 = reinterpret_cast<const float4 *>(bt);
+                    // x = s * qk_scale + bias * log2(e), the bias from this warp's
+                    // slot (columns past Nk hold 0 and are masked below)
+                    const float4 *bt = reinterpret_cast<const float4 *>(bslots + (t & 1) * L::kBiasSlot);
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const float4 bb = __ldg(b4 + c);
-                            x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, bb.x * kLog2e);
-                            x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, bb.y * kLog2e);
-                            x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, bb.z * kLog2e);
-                            x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, bb.w * kLog2e);
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 128; ++c) {
-                            const float bb = (kv0 + c < p.Nk) ? __ldg(bt + c) * kLog2e : 0.f;
-                            x[c] = fmaf(__uint_as_float(sr[c]), qk, bb);
-                        }
+                    for (int c = 0; c < 32; ++c) {
+                        const float4 bb = bt[c];
+                        x[4 * c + 0] = fmaf(__uint_as_float(sr[4 * c + 0]), qk, bb.x);
+                        x[4 * c + 1] = fmaf(__uint_as_float(sr[4 * c + 1]), qk, bb.y);
+                        x[4 * c + 2] = fmaf(__uint_as_float(sr[4 * c + 2]), qk, bb.z);
+                        x[4 * c + 3] = fmaf(__uint_as_float(sr[4 * c + 3]), qk, bb.w);
                     }
                 } else if constexpr (HAS_MASK) {
                     // x = s * qk_scale + M_ij * log2(e); the thread reads its own
@@ -772,6 +804,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // the next unit's first P.V may overwrite O_i only after these loads
             tc_fence_before();
         }
+        if constexpr (HAS_BIAS) cp_async_wait<0>();   // no bias copy outlives the CTA
         named_bar_sync(1, kThreads);
     } else {
         named_bar_sync(1, kThreads);   // idle warps 10, 11
@@ -861,10 +894,11 @@ template <int D, int ELEM, bool CAUSAL, bool HAS_BIAS>
 cudaError_t launch_fwd_t(const FwdTensorMaps &tm, const FwdParams &p, int grid, cudaStream_t stream) {
     using L = FwdLayout<D, ELEM>;
     auto kern = fa_fwd_kernel<D, ELEM, CAUSAL, HAS_BIAS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    constexpr int kSmem = HAS_BIAS ? L::kAlloc : L::kAllocNoBias;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     prof_begin(stream, "fa_fwd_kernel");
-    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     return cudaGetLastError();
@@ -875,10 +909,10 @@ cudaError_t launch_mask_t(const FwdTensorMaps &tm, const FwdParams &p, int grid,
     constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
     using L = FwdLayout<D, kElem>;
     auto kern = fa_fwd_kernel<D, kElem, CAUSAL, false, false, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocNoBias);
     if (e != cudaSuccess) return e;
     prof_begin(stream, "fa_fwd_mask_kernel");
-    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAllocNoBias, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     return cudaGetLastError();
@@ -889,10 +923,10 @@ cudaError_t launch_varlen_t(const FwdTensorMaps &tm, const FwdParams &p, int gri
     constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
     using L = FwdLayout<D, kElem>;
     auto kern = fa_fwd_kernel<D, kElem, CAUSAL, false, false, false, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAllocNoBias);
     if (e != cudaSuccess) return e;
     prof_begin(stream, "fa_fwd_varlen_kernel");
-    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, L::kAllocNoBias, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     return cudaGetLastError();
@@ -903,10 +937,11 @@ cudaError_t launch_split_t(const FwdTensorMaps &tm, const FwdParams &p, int grid
     constexpr int kElem = BF16 ? kElemBF16 : kElemF16;
     using L = FwdLayout<D, kElem>;
     auto kern = fa_fwd_kernel<D, kElem, CAUSAL, HAS_BIAS, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    constexpr int kSmem = HAS_BIAS ? L::kAlloc : L::kAllocNoBias;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     prof_begin(stream, "fa_fwd_split_kernel");
-    kern<<<static_cast<unsigned>(grid), kThreads, L::kAlloc, stream>>>(tm.q, tm.k, tm.v, p);
+    kern<<<static_cast<unsigned>(grid), kThreads, kSmem, stream>>>(tm.q, tm.k, tm.v, p);
     prof_end(stream);
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -150,6 +150,27 @@ __device__ __forceinline__ void tma_store_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Per-thread asynchronous global -> shared copy of `bytes` (4 or 16) bytes, of
+// which the first src_bytes are read and the rest zero-filled (src_bytes 0:
+// nothing is read).  Completion is tracked per thread in commit groups.
+template <int BYTES>
+__device__ __forceinline__ void cp_async_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
+    static_assert(BYTES == 4 || BYTES == 16, "cp.async.ca copies 4, 8 or 16 bytes");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;"
+                 ::"r"(dst), "l"(src), "n"(BYTES), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -47,6 +47,21 @@ def test_key_bias(causal):
     check_forward(2, 2, 256, 260, 128, "f16", causal, seed=4, bias_frac=0.3)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_bias_unaligned_rows(causal):
+    # Nk % 4 != 0: the bias rows of batches b > 0 start off 16-byte boundaries,
+    # and the last key tile is ragged
+    check_forward(3, 2, 200, 301, 64, "bf16", causal, seed=21, bias_frac=0.2)
+    check_forward(2, 2, 129, 333, 128, "f16", causal, seed=22, bias_frac=0.1)
+
+
+def test_key_bias_many_units_per_cta():
+    # more work units than SMs, batches interleaved: the bias staged for one
+    # unit's last tile must not leak into the next unit's first tile
+    check_forward(4, 16, 1024, 1024, 64, "bf16", False, seed=23, bias_frac=0.1)
+    check_forward(3, 8, 768, 1000, 128, "bf16", True, seed=24, bias_frac=0.25)
+
+
 def test_large_scores_rescale():
     # scores spanning hundreds of nats: exercises the lazy max rescale
     check_forward(2, 2, 512, 512, 64, "bf16", False, seed=6, qk_std=8.0, v_dist="uniform")

@@ -56,6 +56,11 @@ def test_split_counts(splits):
 
 def test_key_bias_and_long_queries():
     check(2, 2, 300, 2000, 64, "bf16", False, 5, seed=3, bias_frac=0.1)
+
+
+def test_key_bias_unaligned_rows():
+    # Nk % 4 != 0: bias rows of batches b > 0 start off 16-byte boundaries
+    check(3, 2, 17, 1501, 128, "bf16", True, 4, seed=5, bias_frac=0.2)
     check(1, 2, 520, 1400, 128, "bf16", True, 4, seed=4)
 
 
