@@ -119,15 +119,11 @@ WORKLOAD_TITLES = {"llama": "llama-3-8b layer attention", "bwd": "attention back
 # (S, dP, dV, dK, dQ) are split between the two recompute kernels: the dK/dV
 # kernel does S^T, dP^T, dV, dK (4 of 5 = 2.0x forward); the dQ kernel does dQ
 # (0.5x forward) plus a recomputation of S and dP that is not algorithmic work.
-# When both run as one launch (fa_bwd_grad_kernel) it does all five products
-# (2.5x forward) and executes seven (3.5x).
 KERNEL_FWD_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_fwd_split_kernel": 1.0,
-                       "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5,
-                       "fa_bwd_grad_kernel": 2.5}
+                       "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 0.5}
 # tile products each kernel executes, as multiples of the forward (2 products)
 KERNEL_EXEC_MULTIPLE = {"fa_fwd_kernel": 1.0, "fa_fwd_split_kernel": 1.0,
-                        "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5,
-                        "fa_bwd_grad_kernel": 3.5}
+                        "fa_bwd_dkdv_kernel": 2.0, "fa_bwd_dq_kernel": 1.5}
 
 
 def max_over_ranks(x, world, device=None):
@@ -148,9 +144,11 @@ def weak_scaling_value(world, step_flops, steps, t_max_ms):
 
 
 def kernel_table(records, w):
-    """Per-kernel totals of fa_profile_read() records over the timed steps."""
+    """Per-kernel totals of fa_profile_read() records over the timed steps, with
+    each known kernel's algorithmic TFLOP/s and algorithmic HBM GB/s."""
     from exact_attention_112_b200 import metrics
     f1 = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], w["causal"])
+    elem = 1 if w["dtype"] == "e4m3" else 2
     agg = {}
     for name, ms in records:
         a = agg.setdefault(name, [0, 0.0])
@@ -163,8 +161,30 @@ def kernel_table(records, w):
         if name in KERNEL_FWD_MULTIPLE:
             e["algorithmic_tflops"] = KERNEL_FWD_MULTIPLE[name] * f1 / (ms / n * 1e-3) / 1e12
             e["executed_tflops"] = KERNEL_EXEC_MULTIPLE[name] * f1 / (ms / n * 1e-3) / 1e12
+        nb = metrics.kernel_bytes(name, w["B"], w["H"], w["Nq"], w["Nk"], w["D"], elem=elem,
+                                  bias=w.get("bias_frac", 0) > 0, splits=w.get("splits", 1))
+        if nb is not None:
+            e["algorithmic_bytes"] = nb
+            e["algorithmic_gbs"] = nb / (ms / n * 1e-3) / 1e9
         out[name] = e
     return out
+
+
+def pick_roofline(kd, peak_tflops, hbm_gbs):
+    """The roofline that binds one kernel (a kernel_table entry): HBM when its
+    algorithmic FLOP per byte is below the ridge (peak FLOP/s over peak
+    bytes/s), else the tensor cores; achieved and peak in the bound's unit."""
+    intensity = kd["algorithmic_tflops"] * 1e12 / (kd["algorithmic_gbs"] * 1e9)
+    ridge = peak_tflops * 1e12 / (hbm_gbs * 1e9)
+    if intensity < ridge:
+        r = {"bound": "hbm", "achieved": kd["algorithmic_gbs"], "peak": hbm_gbs, "unit": "GB/s",
+             "frac": kd["algorithmic_gbs"] / hbm_gbs}
+    else:
+        r = {"bound": "tensor", "achieved": kd["algorithmic_tflops"], "peak": peak_tflops, "unit": UNIT,
+             "frac": kd["algorithmic_tflops"] / peak_tflops}
+    r.update({"algorithmic_bytes_per_launch": kd["algorithmic_bytes"], "flop_per_byte": intensity,
+              "ridge_flop_per_byte": ridge})
+    return r
 
 
 def workload_name(w, passes):
@@ -612,10 +632,12 @@ def run_ours(args):
         peak *= 2.0
         peak_source += " x 2 (nominal FP8 / BF16 dense ratio)"
     dom = max((k for k in kernels if k in KERNEL_FWD_MULTIPLE), key=lambda k: kernels[k]["share"])
-    achieved = kernels[dom]["algorithmic_tflops"]
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-            "frac": achieved / peak, "traffic": load_traffic(dom, w), "kernel": dom,
-            "peak_source": peak_source}
+    hbm_peak = float(peaks["hbm_gbs"])
+    roof = pick_roofline(kernels[dom], peak, hbm_peak)
+    roof["peak_source"] = (peak_source if roof["bound"] == "tensor" else
+                           f"{peak_kind} HBM copy bandwidth" +
+                           (" (MEASURED_PEAKS.json)" if peak_kind == "measured" else " 6.65 TB/s"))
+    roof.update({"traffic": load_traffic(dom, w), "kernel": dom})
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,

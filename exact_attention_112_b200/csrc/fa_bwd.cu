@@ -206,36 +206,55 @@ __device__ __forceinline__ int next_ktile(const BwdParams &p, long long plane, i
 }
 
 // ---------------------------------------------------------------------------
-// 1. D_i = rowsum(dO * O).  One warp per row.
+// 1. D_i = rowsum(dO * O).  Each lane reads 16 bytes of a row of O and of dO
+// (D/8 lanes per row, 32/(D/8) rows per warp-wide load) and a warp issues
+// kPreUnroll such loads before it reduces, so that enough bytes are in flight
+// to keep HBM busy; the row sum is a butterfly over the row's lanes.
 // ---------------------------------------------------------------------------
+constexpr int kPreUnroll = 4;
+
+template <bool BF16>
+__device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b) {
+    const float2 a0 = unpack2<BF16>(a.x), a1 = unpack2<BF16>(a.y), a2 = unpack2<BF16>(a.z), a3 = unpack2<BF16>(a.w);
+    const float2 b0 = unpack2<BF16>(b.x), b1 = unpack2<BF16>(b.y), b2 = unpack2<BF16>(b.z), b3 = unpack2<BF16>(b.w);
+    return ((a0.x * b0.x + a0.y * b0.y) + (a1.x * b1.x + a1.y * b1.y)) +
+           ((a2.x * b2.x + a2.y * b2.y) + (a3.x * b3.x + a3.y * b3.y));
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *__restrict__ o,
                                                          const uint16_t *__restrict__ dO,
                                                          float *__restrict__ Di,
                                                          long long rows) {
-    const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    constexpr int kLanes = D / 8;               // 16-byte chunks per row
+    constexpr int kRowsPerLoad = 32 / kLanes;   // rows covered by one warp-wide load
+    constexpr int kRowsPerIter = kRowsPerLoad * kPreUnroll;
     const int lane = threadIdx.x & 31;
+    const int sub = lane / kLanes;              // the lane's row within a load
+    const int chunk = lane % kLanes;            // the lane's 16 bytes within the row
+    const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-    for (long long r = warp_global; r < rows; r += nwarps) {
-        constexpr int kPer = D / 32;   // 16-bit values per lane (2 or 4)
-        const uint16_t *orow = o + r * D + lane * kPer;
-        const uint16_t *drow = dO + r * D + lane * kPer;
-        float acc = 0.f;
-        if constexpr (kPer == 4) {
-            const uint2 a = *reinterpret_cast<const uint2 *>(orow);
-            const uint2 b = *reinterpret_cast<const uint2 *>(drow);
-            const float2 a0 = unpack2<BF16>(a.x), a1 = unpack2<BF16>(a.y);
-            const float2 b0 = unpack2<BF16>(b.x), b1 = unpack2<BF16>(b.y);
-            acc = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
-        } else {
-            const uint32_t a = *reinterpret_cast<const uint32_t *>(orow);
-            const uint32_t b = *reinterpret_cast<const uint32_t *>(drow);
-            const float2 a0 = unpack2<BF16>(a), b0 = unpack2<BF16>(b);
-            acc = a0.x * b0.x + a0.y * b0.y;
+    for (long long r0 = warp_global * kRowsPerIter; r0 < rows; r0 += nwarps * kRowsPerIter) {
+        uint4 a[kPreUnroll], b[kPreUnroll];
+#pragma unroll
+        for (int u = 0; u < kPreUnroll; ++u) {
+            const long long r = r0 + u * kRowsPerLoad + sub;
+            if (r < rows) {
+                a[u] = __ldg(reinterpret_cast<const uint4 *>(o + r * D) + chunk);
+                b[u] = __ldg(reinterpret_cast<const uint4 *>(dO + r * D) + chunk);
+            } else {
+                a[u] = make_uint4(0u, 0u, 0u, 0u);
+                b[u] = a[u];
+            }
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) Di[r] = acc;
+        for (int u = 0; u < kPreUnroll; ++u) {
+            float acc = dot8<BF16>(a[u], b[u]);
+#pragma unroll
+            for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            const long long r = r0 + u * kRowsPerLoad + sub;
+            if (chunk == 0 && r < rows) Di[r] = acc;
+        }
     }
 }
 
@@ -1214,7 +1233,8 @@ template <int D, bool BF16>
 cudaError_t launch_pre(const BwdParams &p, cudaStream_t s) {
     const long long rows = p.cu_q ? static_cast<long long>(p.H) * p.total_q
                                   : static_cast<long long>(p.B) * p.H * p.Nq;
-    const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+    constexpr long long kRowsPerBlock = 8LL * (32 / (D / 8)) * kPreUnroll;   // 8 warps per block
+    const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + kRowsPerBlock - 1) / kRowsPerBlock, 148LL * 8));
     prof_begin(s, "fa_bwd_pre_kernel");
     fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
                                                      static_cast<const uint16_t *>(p.dO), p.Di, rows);
@@ -1243,17 +1263,8 @@ template <int D, bool BF16>
 cudaError_t launch_bwd_d(const BwdTensorMaps &tm, const BwdParams &p, bool causal, bool bias,
                          cudaStream_t s) {
     // 1. D_i
-    {
-        const long long rows = static_cast<long long>(p.B) * p.H * p.Nq;
-        const unsigned grid = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 16));
-        prof_begin(s, "fa_bwd_pre_kernel");
-        fa_bwd_pre_kernel<D, BF16><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(p.o),
-                                                         static_cast<const uint16_t *>(p.dO), p.Di, rows);
-        prof_end(s);
-        note_launch();
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
+    cudaError_t e = launch_pre<D, BF16>(p, s);
+    if (e != cudaSuccess) return e;
     // 2. dK, dV and 3. dQ
     if (causal)
         return bias ? launch_grad_t<D, BF16, true, true>(tm, p, s) : launch_grad_t<D, BF16, true, false>(tm, p, s);

@@ -34,3 +34,27 @@ def bwd_bytes(B, H, Nq, Nk, D, elem=2):
     writes = elem * B * H * D * (Nq + 2 * Nk)
     rowterm = 2 * 4 * B * H * Nq
     return reads + writes + rowterm
+
+
+def kernel_bytes(name, B, H, Nq, Nk, D, elem=2, out_elem=2, bias=False, splits=1):
+    """Algorithmic HBM bytes of one launch of a library kernel (every input
+    byte read once, every output byte written once), or None for a kernel this
+    table does not know.  elem is the byte size of Q, K, V (and dO), out_elem
+    that of O and the gradients; LSE, the row term D_i and split-KV partials
+    are fp32."""
+    BH = B * H
+    qkv = elem * BH * D * (Nq + 2 * Nk)
+    rows = BH * Nq
+    if name == "fa_fwd_kernel":
+        return qkv + out_elem * BH * Nq * D + 4 * rows + (4 * B * Nk if bias else 0)
+    if name == "fa_fwd_split_kernel":
+        return qkv + splits * rows * (4 * D + 4) + (4 * B * Nk if bias else 0)
+    if name == "fa_fwd_combine_kernel":
+        return splits * rows * (4 * D + 4) + out_elem * rows * D + 4 * rows
+    if name == "fa_bwd_pre_kernel":
+        return 2 * out_elem * rows * D + 4 * rows
+    if name == "fa_bwd_dkdv_kernel":
+        return qkv + elem * rows * D + 8 * rows + 2 * out_elem * BH * Nk * D + (4 * B * Nk if bias else 0)
+    if name == "fa_bwd_dq_kernel":
+        return qkv + elem * rows * D + 8 * rows + out_elem * rows * D + (4 * B * Nk if bias else 0)
+    return None

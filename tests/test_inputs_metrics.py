@@ -88,3 +88,48 @@ def test_sample_rows_cover_every_tile_boundary():
         assert t in rows and min(t + 127, 999) in rows
     assert rows[0] == 0 and rows[-1] == 999
     assert np.all(np.diff(rows) > 0)
+
+
+def test_kernel_bytes_add_up_to_the_pass_totals():
+    # the forward kernel's bytes are the forward's; the backward's three kernels
+    # read Q, K, V, dO twice (once per recompute kernel) and O once, and write
+    # dQ, dK, dV once
+    B, H, N, D = 1, 32, 8192, 128
+    assert metrics.kernel_bytes("fa_fwd_kernel", B, H, N, N, D) == metrics.fwd_bytes(B, H, N, N, D)
+    t = 64 * 2 ** 20                  # one [1, 32, 8192, 128] 16-bit tensor
+    rows = 2 ** 20                    # one fp32 value per query row
+    assert metrics.kernel_bytes("fa_bwd_pre_kernel", B, H, N, N, D) == 2 * t + rows
+    assert metrics.kernel_bytes("fa_bwd_dkdv_kernel", B, H, N, N, D) == 6 * t + 2 * rows
+    assert metrics.kernel_bytes("fa_bwd_dq_kernel", B, H, N, N, D) == 5 * t + 2 * rows
+    # fp8 inputs, bf16 output
+    assert metrics.kernel_bytes("fa_fwd_kernel", B, H, N, N, D, elem=1) == 3 * t // 2 + t + rows
+    # split-KV partials: fp32 O_s and LSE_s per split
+    assert metrics.kernel_bytes("fa_fwd_split_kernel", 1, 8, 256, 65536, 128, splits=16) == \
+        2 * (8 * 256 * 128 + 2 * 8 * 65536 * 128) + 16 * 8 * 256 * (4 * 128 + 4)
+    assert metrics.kernel_bytes("fa_unknown_kernel", B, H, N, N, D) is None
+
+
+def test_roofline_picks_the_binding_bound():
+    import bench
+    # Llama forward: ~2000 FLOP/byte, far above the ridge (~239) -> tensor
+    w = inputs.workload("llama")
+    f = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], True)
+    nb = metrics.kernel_bytes("fa_fwd_kernel", w["B"], w["H"], w["Nq"], w["Nk"], w["D"])
+    ms = 0.47
+    kd = {"algorithmic_tflops": f / (ms * 1e-3) / 1e12, "algorithmic_gbs": nb / (ms * 1e-3) / 1e9,
+          "algorithmic_bytes": nb}
+    r = bench.pick_roofline(kd, 1590.0, 6650.0)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["frac"] == pytest.approx(f / (ms * 1e-3) / 1e12 / 1590.0)
+    assert r["flop_per_byte"] == pytest.approx(f / nb)
+    # sequence sweep at N = 512, causal: ~128 FLOP/byte, below the ridge -> HBM
+    w = inputs.workload("sweep", N=512)
+    f = metrics.fwd_flops(w["B"], w["H"], w["Nq"], w["Nk"], w["D"], True)
+    nb = metrics.kernel_bytes("fa_fwd_kernel", w["B"], w["H"], w["Nq"], w["Nk"], w["D"])
+    ms = 0.08
+    kd = {"algorithmic_tflops": f / (ms * 1e-3) / 1e12, "algorithmic_gbs": nb / (ms * 1e-3) / 1e9,
+          "algorithmic_bytes": nb}
+    r = bench.pick_roofline(kd, 1590.0, 6650.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6650.0
+    assert r["achieved"] == pytest.approx(nb / 0.08e-3 / 1e9)
+    assert r["ridge_flop_per_byte"] == pytest.approx(1590e12 / 6650e9)
