@@ -347,10 +347,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     q_issued = i + 1;
                 }
                 if (!ok) break;
-                {   // warm L2 with the next unit's Q tiles
+                {   // warm L2 with the next unit's Q tiles while this unit runs; a
+                    // unit of fewer than 8 key tiles does without (measured: the
+                    // prefetch then delays more than it hides)
                     int r2 = r + 1;
                     Unit nx;
-                    if (next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r2, nx))
+                    if (w.n_kv >= 8 && next_work<CAUSAL, SPLIT, VARLEN, HAS_MASK>(p, r2, nx))
                         for (int i = 0; i < 2; ++i)
                             for (int c = 0; c < L::kChunks; ++c)
                                 tma_prefetch_l2_3d(&tm_q, c * L::kChunkElems, nx.q_y0 + nx.m0 + i * kBM, nx.z);
