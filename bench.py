@@ -67,7 +67,8 @@ def parse_args(argv=None):
                     help="override the workload's head count (smaller profiling cases)")
     ap.add_argument("--splits", type=int, default=None,
                     help="forward through fa_fwd_splitkv with this many key ranges "
-                         "(default 16 for the decode workload, else the single-pass fa_fwd)")
+                         "(default: fa_splitkv_num_splits for the decode workload, else the "
+                         "single-pass fa_fwd)")
     return ap.parse_args(argv)
 
 
@@ -95,7 +96,16 @@ def workload_cfg(args):
     if args.seq_len is not None or args.causal is not None or args.heads is not None:
         # keeps stored ncu traffic (keyed by workload name) off modified shapes
         w["name"] = f"{w['name']}-H{w['H']}-N{w['Nq']}-{'causal' if w['causal'] else 'full'}"
-    w["splits"] = args.splits if args.splits is not None else (16 if args.workload == "decode" else 1)
+    if args.splits is not None:
+        w["splits"] = args.splits
+    elif args.workload == "decode":
+        # the library's own choice for these sizes and this device's SM count
+        import torch
+        import exact_attention_112_b200 as fa
+        sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+        w["splits"] = fa.fa_splitkv_num_splits(w["B"], w["H"], w["Nq"], w["Nk"], sms)
+    else:
+        w["splits"] = 1
     return w
 
 

@@ -24,7 +24,7 @@ __all__ = [
     "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_ERR_INTERNAL", "FA_F16", "FA_BF16", "FaError",
     "lib", "library_path", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes",
     "fa_bwd_noalloc",
-    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_mask", "fa_bwd_mask",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_splitkv_num_splits", "fa_fwd_mask", "fa_bwd_mask",
     "fa_fwd_varlen", "fa_bwd_varlen", "fa_mask_tile_flags_bytes", "mask_tile_flags",
     "FA_BWD_NOALLOC_MAX_ROWS",
     "fa_status_string", "fa_device_status", "fa_debug_wait_timeout", "fa_launch_count",
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
             L.fa_bwd_varlen.restype = i
             L.fa_fwd_splitkv_workspace_bytes.argtypes = [i, i, i, i, i, i]
             L.fa_fwd_splitkv_workspace_bytes.restype = sz
+            L.fa_splitkv_num_splits.argtypes = [i, i, i, i, i]
+            L.fa_splitkv_num_splits.restype = i
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
             L.fa_fwd_splitkv.restype = i
             L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -393,6 +395,12 @@ def fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, workspace, cu_seqlens_q, cu_s
 
 def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits) -> int:
     return int(lib().fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, D, num_splits))
+
+
+def fa_splitkv_num_splits(B, H, Nq, Nk, num_sms=0) -> int:
+    """A num_splits for fa_fwd_splitkv on these sizes (num_sms 0: the current
+    device's SM count)."""
+    return int(lib().fa_splitkv_num_splits(B, H, Nq, Nk, num_sms))
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, num_splits, workspace, causal=False, scale=None,

@@ -470,6 +470,35 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_splitkv_num_splits(int B, int H, int Nq, int Nk, int num_sms) {
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || num_sms < 0) return 1;
+    if (num_sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms < 1) {
+            cudaGetLastError();
+            return 1;
+        }
+    }
+    const long long units = static_cast<long long>(B) * H * ((Nq + 255) / 256);
+    const int tiles = (Nk + 127) / 128;
+    if (units >= num_sms || tiles < 2) return 1;
+    long long best_cost = -1;
+    int best = 1;
+    for (int s = 1; s <= std::min(tiles, 256); ++s) {
+        const int per = (tiles + s - 1) / s;          // key tiles per split
+        const int used = (tiles + per - 1) / per;     // splits that hold tiles
+        if (used != s) continue;                      // the same cut as a smaller count
+        const long long waves = (units * s + num_sms - 1) / num_sms;
+        const long long cost = waves * (per + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int D) {
     (void)Nk;
     if (B < 1 || H < 1 || Nq < 0 || (D != 64 && D != 128)) return 0;

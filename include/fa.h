@@ -114,6 +114,19 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
  * A split whose keys are all masked for a row contributes LSE_s = -inf.
  */
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int D, int num_splits);
+
+/*
+ * A num_splits for fa_fwd_splitkv() on these sizes (host arithmetic only, no
+ * device call unless num_sms is 0).  The forward runs units of 256 query rows
+ * per (b, h); with few units the SMs idle, and splitting the keys multiplies
+ * the units.  The count minimises waves * (key tiles per split + 1), where
+ * waves = ceil(units * splits / num_sms) and the +1 charges each unit's fixed
+ * cost (Q load, pipeline fill, partial write) as one key tile; ties go to
+ * fewer splits.  Returns 1 when the units already fill the SMs, when there is
+ * a single key tile, or for invalid sizes.  num_sms: the device's SM count,
+ * or 0 for that of the current device (148 on B200).
+ */
+int fa_splitkv_num_splits(int B, int H, int Nq, int Nk, int num_sms);
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int H, int Nq, int Nk, int D, int causal, float scale,
                    int dtype, const float *key_bias, int num_splits, void *workspace,

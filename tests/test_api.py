@@ -339,3 +339,25 @@ def test_mask_tile_flags_arguments(L):
     assert call(nbytes=5) == fa.FA_ERR_INVALID_ARG         # 3 x 2 tiles need 6 bytes
     assert call(Bm=0) == fa.FA_ERR_INVALID_ARG
     assert call(Nq=0, mask=None, flags=None) == fa.FA_OK   # no tile: nothing to do
+
+
+def test_splitkv_num_splits_choice():
+    # host arithmetic only (an explicit SM count touches no device)
+    import exact_attention_112_b200 as fa
+    # 8 units of 256 rows over 512 key tiles on 148 SMs: 18 splits of 29 tiles
+    # fill 144 SMs in one wave (16 splits would leave 20 SMs idle)
+    assert fa.fa_splitkv_num_splits(1, 8, 256, 65536, 148) == 18
+    assert fa.fa_splitkv_num_splits(1, 8, 1, 65536, 148) == 18
+    # enough units already: no split
+    assert fa.fa_splitkv_num_splits(1, 32, 8192, 8192, 148) == 1
+    # a single key tile cannot be split
+    assert fa.fa_splitkv_num_splits(1, 1, 1, 100, 148) == 1
+    # invalid sizes
+    assert fa.fa_splitkv_num_splits(0, 8, 256, 65536, 148) == 1
+    assert fa.fa_splitkv_num_splits(1, 8, 256, 65536, -1) == 1
+    # every split holds key tiles, and the waves fit the SM count
+    for B, H, Nq, Nk in [(1, 1, 1, 1000), (2, 4, 64, 20000), (1, 16, 512, 131072), (3, 5, 300, 7777)]:
+        s = fa.fa_splitkv_num_splits(B, H, Nq, Nk, 148)
+        tiles = (Nk + 127) // 128
+        per = -(-tiles // s)
+        assert 1 <= s <= min(256, tiles) and -(-tiles // per) == s
