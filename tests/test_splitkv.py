@@ -90,3 +90,13 @@ def test_argument_errors():
         with pytest.raises(fa.FaError) as e:
             fa.fa_fwd_splitkv(q, k, k, o, lse, bad, ws)
         assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_library_split_count(causal):
+    # the count fa_splitkv_num_splits picks for a decoding shape on this GPU
+    # (one query block of 8 heads over 16384 keys: more splits than SMs/units)
+    B, H, Nq, Nk, D = 1, 8, 64, 16384, 128
+    s = fa.fa_splitkv_num_splits(B, H, Nq, Nk)
+    assert 1 < s <= 256
+    check(B, H, Nq, Nk, D, "bf16", causal, s, seed=77)
