@@ -822,25 +822,57 @@ __global__ void __launch_bounds__(256) fa_fwd_combine_kernel(const float *__rest
                                                              uint16_t *__restrict__ o, float *__restrict__ lse,
                                                              long long rows, int num_splits) {
     constexpr int kPer = D / 32;   // values per lane (2 or 4)
+    constexpr int kU = 4;          // O_s rows in flight per lane
     const int lane = threadIdx.x & 31;
     const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
     for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+        // m = max_s LSE_s, the lanes taking the splits in turn
         float m = neg_inf();
-        for (int s = 0; s < num_splits; ++s) m = fmaxf(m, lse_part[s * rows + r]);
+        for (int sp = lane; sp < num_splits; sp += 32) m = fmaxf(m, lse_part[sp * rows + r]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         float acc[kPer];
 #pragma unroll
         for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
         float wsum = 0.f;
         if (m != neg_inf()) {
-            for (int s = 0; s < num_splits; ++s) {
-                const float ls = lse_part[s * rows + r];
-                if (ls == neg_inf()) continue;
-                const float w = __expf(ls - m);
-                wsum += w;
-                const float *src = o_part + (s * rows + r) * D + lane * kPer;
+            for (int s0 = 0; s0 < num_splits; s0 += 32) {
+                // lane k holds the weight of split s0 + k; every lane sums the
+                // weighted O_s rows of the chunk, kU loads in flight
+                float wl = 0.f;
+                if (s0 + lane < num_splits) {
+                    const float ls = lse_part[(s0 + lane) * rows + r];
+                    wl = ls == neg_inf() ? 0.f : __expf(ls - m);
+                }
+                wsum += wl;
+                const int cnt = min(32, num_splits - s0);
+                for (int k = 0; k < cnt; k += kU) {
+                    float w[kU], v[kU][kPer];
 #pragma unroll
-                for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+                    for (int u = 0; u < kU; ++u) {
+                        w[u] = __shfl_sync(0xffffffffu, wl, (k + u) & 31);
+                        const int sp = s0 + min(k + u, cnt - 1);
+                        const float *src = o_part + (sp * rows + r) * D + lane * kPer;
+                        if constexpr (kPer == 4) {
+                            const float4 t4 = *reinterpret_cast<const float4 *>(src);
+                            v[u][0] = t4.x; v[u][1] = t4.y; v[u][2] = t4.z; v[u][3] = t4.w;
+                        } else {
+                            const float2 t2 = *reinterpret_cast<const float2 *>(src);
+                            v[u][0] = t2.x; v[u][1] = t2.y;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        // a split that saw no key (weight 0) adds nothing, whatever its row holds
+                        if (k + u < cnt && w[u] != 0.f) {
+#pragma unroll
+                            for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
+                        }
+                    }
+                }
             }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
         }
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
         uint32_t packed[kPer / 2];
