@@ -699,7 +699,8 @@ def load_traffic(kernel, w):
 
 # The source file that defines each kernel; its revision also covers the
 # device headers every kernel file includes.
-KERNEL_SOURCE = {"fa_fwd_kernel": "fa_fwd.cu", "fa_bwd_dkdv_kernel": "fa_bwd.cu",
+KERNEL_SOURCE = {"fa_fwd_kernel": "fa_fwd.cu", "fa_fwd_split_kernel": "fa_fwd.cu",
+                 "fa_fwd_combine_kernel": "fa_fwd.cu", "fa_bwd_dkdv_kernel": "fa_bwd.cu",
                  "fa_bwd_dq_kernel": "fa_bwd.cu", "fa_bwd_pre_kernel": "fa_bwd.cu"}
 DEVICE_HEADERS = ("fa_ptx.cuh", "fa_internal.h")
 
