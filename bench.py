@@ -96,6 +96,9 @@ def workload_cfg(args):
     if args.seq_len is not None or args.causal is not None or args.heads is not None:
         # keeps stored ncu traffic (keyed by workload name) off modified shapes
         w["name"] = f"{w['name']}-H{w['H']}-N{w['Nq']}-{'causal' if w['causal'] else 'full'}"
+    # stored ncu traffic is looked up by this key; 8-bit inputs move other byte
+    # counts than the 16-bit captures
+    w["traffic_key"] = w["name"] + ("-e4m3" if w["dtype"] == "e4m3" else "")
     if args.splits is not None:
         w["splits"] = args.splits
     elif args.workload == "decode":
@@ -689,7 +692,7 @@ def load_traffic(kernel, w):
         return None
     try:
         d = json.load(open(path))
-        ent = d.get(f"{kernel}:{w['name']}")
+        ent = d.get(f"{kernel}:{w.get('traffic_key', w['name'])}")
         if ent and ent.get("kernel_rev") == kernel_rev(kernel):
             return ent["bytes_per_launch"]
     except (OSError, ValueError):
