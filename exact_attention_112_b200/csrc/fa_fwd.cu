@@ -43,7 +43,8 @@
 //     = e^(s - m_new): l, o and the final LSE all use the same m_ref.
 //   * Causal: key tiles entirely above the diagonal are never loaded or
 //     multiplied; tiles crossing it are masked per element.
-//   * Additive terms after scaling: a per-key bias [B, Nk] (broadcast loads),
+//   * Additive terms after scaling: a per-key bias [B, Nk] (copied one key
+//     tile ahead into a shared-memory slot per warp and read as broadcasts),
 //     or a general mask [B or 1, H or 1, Nq, Nk] whose row each softmax
 //     thread reads itself (the "+ mask" of the SDPA formula in full).
 //   * Epilogue: each softmax thread divides its O row by l and stores it
