@@ -398,7 +398,20 @@ def cpu_baseline(w, target_s, passes, gpu=None):
                                       w["causal"], 1.0 / math.sqrt(w["D"]), rows=rows)
     base = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": sample_text(w, rows, passes) + f" ({fl / 1e9:.1f} GFLOP algorithmic, {dt:.1f} s)",
-            "seconds": dt}
+            "seconds": dt,
+            # query rows (of every (b, h)) per second, and the whole step's time
+            # at the sample's FLOP rate
+            "rows_per_s": len(rows) * w["B"] * w["H"] / dt,
+            "full_step_s_extrapolated": sum(flops_of(w, passes).values()) / (fl / dt)}
+    if w.get("name") == "tiny":
+        # the single-thread figure beside the all-core one (the tiny workload
+        # is small enough to time whole)
+        oracle.set_threads(1)
+        try:
+            dt1, fl1 = oracle_rows_time(arrs, w, rows, passes)
+        finally:
+            oracle.set_threads(cores)
+        base["one_thread"] = {"value": fl1 / dt1 / 1e12, "seconds": dt1}
     if gpu is None:
         return base, None
     gpu = dict(gpu)

@@ -50,3 +50,17 @@ def test_planted_errors_fail(case, what):
         t[0, 1] *= 1.1                          # dV of one head scaled
     rep = bench.parity_report(w, rows, ref, bad)
     assert not rep["ok"], (what, rep)
+
+
+def test_cpu_baseline_fields():
+    """The cpu_baseline leg reports its FLOP rate, the rows per second and the
+    whole step's extrapolated time (consistent with each other), and for the
+    tiny workload a single-thread figure as well."""
+    w = inputs.workload("tiny")
+    base, report = bench.cpu_baseline(w, 0.2, ["fwd"])
+    assert report is None
+    total = sum(bench.flops_of(w, ["fwd"]).values())
+    assert base["value"] > 0 and base["rows_per_s"] > 0 and base["cores"] >= 1
+    assert math.isclose(base["full_step_s_extrapolated"] * base["value"] * 1e12, total, rel_tol=1e-9)
+    assert base["one_thread"]["value"] > 0 and base["one_thread"]["seconds"] > 0
+    assert oracle.max_threads() == base["cores"]   # the thread count is restored
