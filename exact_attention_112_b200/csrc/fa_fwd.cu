@@ -139,6 +139,16 @@ struct FwdLayout {
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
+// 32 bytes to global memory in one 256-bit store (sm_100); `p` must be 32-byte
+// aligned.  A row-per-thread store then fills whole 32-byte sectors instead of
+// halves of two.
+__device__ __forceinline__ void st_global_v8(void *p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1),
+                 "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+
 // Two fp32 values -> one 32-bit word of two 16-bit values (lo in the low half).
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -539,6 +549,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t tS = tl + (i ? L::kColS1 : L::kColS0);
         const uint32_t tO = tl + (i ? L::kColO1 : L::kColO0);
         const float qk = p.qk_scale_log2;
+        // O rows start on 128-byte multiples of the base: 256-bit stores when
+        // the base is 32-byte aligned (the library asks for 16 only)
+        const bool o_v8 = (reinterpret_cast<uintptr_t>(p.o) & 31) == 0;
         // Key bias: every row of a tile adds the same 128 values.  Each warp
         // copies them (cp.async, four per lane) into its own shared-memory slot
         // one tile ahead, scales them by log2(e) in place when the tile starts,
@@ -797,9 +810,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         pk[e] = pack2<kOutBF16>(__uint_as_float(orr[2 * e]) * inv_l,
                                                 __uint_as_float(orr[2 * e + 1]) * inv_l);
                     if (qrow < w.len_q) {
+                        if (o_v8) {
+                            // whole 32-byte sectors per store instruction
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                            for (int h8 = 0; h8 < 2; ++h8)
+                                st_global_v8(dst + cc * 4 + 2 * h8, pk[8 * h8], pk[8 * h8 + 1], pk[8 * h8 + 2],
+                                             pk[8 * h8 + 3], pk[8 * h8 + 4], pk[8 * h8 + 5], pk[8 * h8 + 6],
+                                             pk[8 * h8 + 7]);
+                        } else {
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                dst[cc * 4 + q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                        }
                     }
                 }
                 if (qrow < w.len_q) p.lse[w.o_row0 + qrow] = lse;

@@ -37,6 +37,32 @@ def test_edge_sizes(Nq, Nk, causal):
     check_forward(1, 2, Nq, Nk, 64, "bf16", causal, seed=Nq * 1000 + Nk)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_output_base_16_byte_aligned(D):
+    """O whose base is 16- but not 32-byte aligned (a view 16 bytes into a
+    larger buffer) takes the 16-byte store path; the result is bit-identical
+    to the same call with a 32-byte aligned O, and matches the oracle."""
+    B, H, N = 1, 3, 300
+    inp = inputs.make_inputs(B, H, N, N, D, dtype="bf16", seed=77)
+    dev = torch.device("cuda")
+    q, k, v = (inp[x].to(dev) for x in "qkv")
+    o_ref = torch.empty_like(q)
+    lse_ref = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    fa.fa_fwd(q, k, v, o_ref, lse_ref, causal=True)
+    buf = torch.empty(q.numel() + 8, dtype=q.dtype, device=dev)
+    o = buf[8:].view(q.shape)
+    assert o.data_ptr() % 32 == 16
+    lse = torch.empty_like(lse_ref)
+    fa.fa_fwd(q, k, v, o, lse, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    f = inputs.to_f64
+    ref_o, ref_lse = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), None, True, 1.0 / math.sqrt(D))
+    assert float(np.abs(o.float().cpu().numpy() - ref_o).max()) <= TOL_O["bf16"]
+    assert float(np.abs(lse.cpu().numpy() - ref_lse).max()) <= 1e-3
+
+
 def test_many_units_and_heads():
     check_forward(3, 5, 1024, 1024, 128, "bf16", True, seed=5)
 
