@@ -133,3 +133,23 @@ def test_roofline_picks_the_binding_bound():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6650.0
     assert r["achieved"] == pytest.approx(nb / 0.08e-3 / 1e9)
     assert r["ridge_flop_per_byte"] == pytest.approx(1590e12 / 6650e9)
+
+
+def test_traffic_records_are_consistent():
+    """profiles/traffic.json: every entry names an existing ncu summary and holds
+    read + write = bytes_per_launch; the headline's dominant kernel (dK/dV on the
+    Llama workload) has a record for the current sources, so the headline bench
+    line reports `traffic`."""
+    import json
+    import os
+    import bench
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    t = json.load(open(os.path.join(root, "profiles", "traffic.json")))
+    for key, ent in t.items():
+        kernel, _, workload = key.partition(":")
+        assert kernel in bench.KERNEL_SOURCE and workload, key
+        assert ent["read_bytes"] + ent["write_bytes"] == ent["bytes_per_launch"], key
+        src = ent["source"].split(" ")[0]
+        assert src.startswith("profiles/") and os.path.exists(os.path.join(root, src)), (key, src)
+    w = bench.workload_cfg(bench.parse_args([]))
+    assert bench.load_traffic("fa_bwd_dkdv_kernel", w) == t["fa_bwd_dkdv_kernel:llama"]["bytes_per_launch"]
